@@ -1,0 +1,568 @@
+"""CPU oracle of the DraftAttention2 hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only `tests/`, `__graft_entry__.smoke()` and `bench.py`'s cpu_baseline / reference leg
+use this module. It shares no code with the CUDA library.
+
+Sources (cited by page title and section):
+  [DA2]  "DraftAttention2: Fast Video Diffusion with Low-Resolution-Guided Mixed-Precision
+         Attention" (arXiv 2609.32628), Abstract.
+  [DA1]  "DraftAttention: Fast Video Diffusion via Low-Resolution Attention Guidance"
+         (arXiv 2505.14708), Abstract.
+  [NEWS] News article on DraftAttention (szmaozhuayin.com), method overview steps 1-4 and
+         the theoretical-analysis paragraph.
+
+The pages print no equations; where a step is left open the plainest reading is taken
+and listed in the repository's design notes. Every step below is a separate function
+returning its own arrays so that each can be compared with the CUDA path on its own.
+
+Numerics. Floating point is fp64 except where a step is defined in fp32 so that the
+CUDA path can reproduce it bit for bit: the pooled averages (an fp32 running sum in slot
+order, then an IEEE fp32 divide), the operand scales and the operand quantisers (IEEE
+fp32 multiplies/divides, then round-to-nearest-even onto the E4M3 / E2M1 grids).
+
+Parity pins: every function is pinned by `tests/test_oracle_*.py` against closed forms,
+library routines or brute force; the error-decomposition formula itself is not printed
+on the pages (parity unpinned, see `error_decomposition`).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+F32 = np.float32
+E4M3_MAX = 448.0        # largest finite E4M3 value (OCP FP8, bias 7, no infinities)
+E2M1_MAX = 6.0          # largest E2M1 value
+TAG_SKIP, TAG_FP4, TAG_FP8 = 0, 1, 2
+
+
+# ----------------------------------------------------------------------------------------
+# Geometry: windows, blocks, budgets
+# ----------------------------------------------------------------------------------------
+@dataclass(frozen=True)
+class Geometry:
+    B: int
+    H: int
+    d: int
+    F: int
+    Hf: int
+    Wf: int
+    ph: int
+    pw: int
+    ny: int
+    nx: int
+    N: int        # blocks (windows) per (b, h)
+    bs: int       # tokens per block, ph * pw
+    T: int        # valid tokens
+    Tp: int       # padded tokens N * bs
+    n8: int       # FP8 blocks per query block
+    n4: int       # FP4 blocks per query block
+    sm_scale: float
+
+
+def budget_counts(N: int, pct_fp8: int, pct_fp4: int) -> tuple[int, int]:
+    """Blocks kept at FP8 and FP4 per query block: integer percent, rounded half up.
+
+    [DA2] Abstract: the ranking runs under configurable budgets. Reading: the budgets are
+    percentages of the N KV blocks; n8 = floor((p8 N + 50)/100), nk = floor(((p8+p4) N
+    + 50)/100), n4 = nk - n8.
+    """
+    n8 = (pct_fp8 * N + 50) // 100
+    nk = ((pct_fp8 + pct_fp4) * N + 50) // 100
+    return n8, nk - n8
+
+
+def geometry(w) -> Geometry:
+    ny, nx = -(-w.Hf // w.ph), -(-w.Wf // w.pw)
+    N = w.F * ny * nx
+    bs = w.ph * w.pw
+    n8, n4 = budget_counts(N, w.pct_fp8, w.pct_fp4)
+    sm = getattr(w, "sm_scale", 0.0) or 1.0 / math.sqrt(w.d)
+    return Geometry(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, ny, nx, N, bs,
+                    w.F * w.Hf * w.Wf, N * bs, n8, n4, sm)
+
+
+def token_block_slot(g: Geometry):
+    """Block n and slot s of every token t (frame-major t = f Hf Wf + y Wf + x).
+
+    [DA1] Abstract and [NEWS] step 4: tokens are reordered so that each pooled region is
+    one contiguous block. Block n = f ny nx + (y // ph) nx + (x // pw); slot
+    s = (y % ph) pw + (x % pw).
+    """
+    t = np.arange(g.T)
+    f, rem = np.divmod(t, g.Hf * g.Wf)
+    y, x = np.divmod(rem, g.Wf)
+    blk = f * g.ny * g.nx + (y // g.ph) * g.nx + (x // g.pw)
+    slot = (y % g.ph) * g.pw + (x % g.pw)
+    return blk, slot
+
+
+def block_valid(g: Geometry) -> np.ndarray:
+    """[N, bs] bool: slot holds a real token (edge windows are padded)."""
+    blk, slot = token_block_slot(g)
+    valid = np.zeros((g.N, g.bs), dtype=bool)
+    valid[blk, slot] = True
+    return valid
+
+
+def block_counts(g: Geometry) -> np.ndarray:
+    return block_valid(g).sum(axis=1)
+
+
+def permute(x: np.ndarray, g: Geometry) -> np.ndarray:
+    """[B, H, T, d] -> [B, H, N, bs, d]; padded slots hold zeros."""
+    blk, slot = token_block_slot(g)
+    out = np.zeros(x.shape[:2] + (g.N, g.bs) + x.shape[3:], dtype=x.dtype)
+    out[:, :, blk, slot] = x
+    return out
+
+
+def inverse_permute(xp: np.ndarray, g: Geometry) -> np.ndarray:
+    """[B, H, N, bs, d] -> [B, H, T, d]: restore the original token order ([DA1] Abstract)."""
+    blk, slot = token_block_slot(g)
+    return xp[:, :, blk, slot]
+
+
+# ----------------------------------------------------------------------------------------
+# Pooling ([DA2] Abstract: spatial 2D average- and max-pooled queries and keys;
+#          [NEWS] step 1: per-frame spatial downsampling into draft Q/K)
+# ----------------------------------------------------------------------------------------
+def pool(xp: np.ndarray, valid: np.ndarray):
+    """Average and max of each window over its valid tokens, per channel.
+
+    avg: fp32 running sum over the valid slots in increasing slot order, then an IEEE
+    fp32 divide by the number of valid tokens. max: exact. Both fp32 [B, H, N, d].
+    """
+    x = xp.astype(F32)
+    B, H, N, bs, d = x.shape
+    acc = np.zeros((B, H, N, d), dtype=F32)
+    for s in range(bs):
+        take = valid[:, s][None, None, :, None]
+        acc = np.where(take, (acc + x[:, :, :, s, :]).astype(F32), acc)
+    cnt = valid.sum(axis=1).astype(F32)
+    avg = (acc / cnt[None, None, :, None]).astype(F32)
+    xm = np.where(valid[None, None, :, :, None], x, F32(-np.inf))
+    mx = xm.max(axis=3).astype(F32)
+    return avg, mx
+
+
+# ----------------------------------------------------------------------------------------
+# Quantisers: E4M3 (OCP FP8, bias 7, max 448, no inf) and E2M1 (values 0, .5, 1, 1.5, 2,
+# 3, 4, 6), round to nearest with ties to even, saturating to the largest finite value.
+# ----------------------------------------------------------------------------------------
+def e4m3_round(y) -> np.ndarray:
+    """Nearest E4M3 value (fp64), ties to even mantissa, saturating at +-448."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    _, e = np.frexp(a)                                  # a = m 2^e, m in [0.5, 1)
+    quantum = np.where(a >= 2.0 ** -6, np.ldexp(1.0, e - 4), 2.0 ** -9)
+    r = np.minimum(np.rint(a / quantum) * quantum, E4M3_MAX)
+    return np.copysign(r, y)
+
+
+def e4m3_code(y) -> np.ndarray:
+    """E4M3 byte of the nearest value: sign | exponent field (4 bits) | mantissa (3 bits)."""
+    v = e4m3_round(y)
+    a = np.abs(v)
+    _, e = np.frexp(a)
+    normal = a >= 2.0 ** -6
+    ef = np.where(normal, e - 1 + 7, 0)
+    man = np.where(normal, np.rint(np.ldexp(a, -(e - 1)) * 8 - 8), np.rint(a / 2.0 ** -9))
+    code = (ef.astype(np.int64) << 3) | man.astype(np.int64)
+    code = code | (np.signbit(v).astype(np.int64) << 7)
+    return code.astype(np.uint8)
+
+
+def e4m3_decode(code) -> np.ndarray:
+    c = np.asarray(code, dtype=np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    ef = (c >> 3) & 0xF
+    man = c & 7
+    mag = np.where(ef == 0, man * 2.0 ** -9, np.ldexp(1.0 + man / 8.0, ef - 7))
+    return s * mag
+
+
+_E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e2m1_round(y) -> np.ndarray:
+    """Nearest E2M1 value (fp64), ties to even mantissa, saturating at +-6."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    quantum = np.where(a < 2.0, 0.5, np.where(a < 4.0, 1.0, 2.0))
+    r = np.minimum(np.rint(a / quantum) * quantum, E2M1_MAX)
+    return np.copysign(r, y)
+
+
+def e2m1_code(y) -> np.ndarray:
+    """4-bit E2M1 code (sign bit 3, then 2 exponent bits, 1 mantissa bit)."""
+    v = e2m1_round(y)
+    idx = np.searchsorted(_E2M1_GRID, np.abs(v))
+    return (idx | (np.signbit(v).astype(np.int64) << 3)).astype(np.uint8)
+
+
+def e2m1_decode(code) -> np.ndarray:
+    c = np.asarray(code, dtype=np.int64)
+    return np.where(c & 8, -1.0, 1.0) * _E2M1_GRID[c & 7]
+
+
+# ----------------------------------------------------------------------------------------
+# Operand quantisation ([DA2] Abstract: fused operand preparation producing the 8-bit and
+# 4-bit copies used by the mixed-precision kernel). Formats: FP8 E4M3 with an fp32 outer
+# scale; NVFP4-style E2M1 with one E4M3 scale per 16 consecutive elements along the
+# contraction axis and the same fp32 outer scale.
+# ----------------------------------------------------------------------------------------
+def outer_scale(amax):
+    """(s, inv) per group: s = amax/448 (dequantisation), inv = 448/amax (quantisation),
+    both IEEE fp32; s = inv = 1 where amax == 0."""
+    amax = np.asarray(amax, dtype=F32)
+    safe = np.where(amax > 0, amax, F32(1))
+    s = np.where(amax > 0, (safe / F32(E4M3_MAX)).astype(F32), F32(1)).astype(F32)
+    inv = np.where(amax > 0, (F32(E4M3_MAX) / safe).astype(F32), F32(1)).astype(F32)
+    return s, inv
+
+
+def fp4_groups(y: np.ndarray):
+    """y fp32 [..., K] (K % 16 == 0), already divided by its outer scale.
+
+    Group scale sigma = E4M3(amax16 / 6) (IEEE fp32 divide, then RNE); codes =
+    E2M1(y * (1/sigma)) with 1/sigma an IEEE fp32 reciprocal; a group whose sigma is 0
+    is all zero codes. Returns (codes uint8 [..., K], sigma codes uint8 [..., K/16]).
+    """
+    y = y.astype(F32)
+    sh = y.shape
+    yg = y.reshape(sh[:-1] + (sh[-1] // 16, 16))
+    amax16 = np.abs(yg).max(axis=-1).astype(F32)
+    sig_code = e4m3_code((amax16 / F32(E2M1_MAX)).astype(F32))
+    sig = e4m3_decode(sig_code).astype(F32)
+    rcp = np.where(sig > 0, (F32(1) / np.where(sig > 0, sig, F32(1))).astype(F32), F32(0))
+    z = (yg * rcp[..., None]).astype(F32)
+    codes = np.where(sig[..., None] > 0, e2m1_code(z), np.uint8(0)).astype(np.uint8)
+    return codes.reshape(sh), sig_code
+
+
+def fp4_dequant(codes, sig_code) -> np.ndarray:
+    """Values sigma * e2m1 (fp64), without the outer scale."""
+    v = e2m1_decode(codes)
+    sh = v.shape
+    vg = v.reshape(sh[:-1] + (sh[-1] // 16, 16)) * e4m3_decode(sig_code)[..., None]
+    return vg.reshape(sh)
+
+
+def quantise_qk(xp: np.ndarray, valid: np.ndarray):
+    """Q or K, per (b, h, block) outer scale from the block amax.
+
+    xp: [B, H, N, bs, d] (padded slots zero). Returns dict with
+      s    fp32 [B,H,N]       dequantisation scale amax/448
+      q8   uint8 [B,H,N,bs,d] E4M3 codes of x * (448/amax)
+      q4   uint8 [B,H,N,bs,d] E2M1 codes (one per element, unpacked)
+      sf4  uint8 [B,H,N,bs,d/16] E4M3 group scales along d
+    """
+    x = xp.astype(F32)
+    amax = np.abs(x).max(axis=(3, 4)).astype(F32)
+    s, inv = outer_scale(amax)
+    y = (x * inv[..., None, None]).astype(F32)
+    q8 = e4m3_code(y)
+    q4, sf4 = fp4_groups(y)
+    return dict(s=s, q8=q8, q4=q4, sf4=sf4)
+
+
+def v_channel_amax(v: np.ndarray) -> np.ndarray:
+    """amax of V over all tokens, per (b, h, channel): fp32 [B, H, d]."""
+    return np.abs(v.astype(F32)).max(axis=2).astype(F32)
+
+
+def quantise_v(vp: np.ndarray, amax_c: np.ndarray):
+    """V, per (b, h, channel) outer scale (it must factor out of the P V sum over tokens).
+
+    Groups of 16 run along tokens (the P V contraction axis) within a block.
+    Returns s fp32 [B,H,d], q8 uint8 [B,H,N,bs,d], q4 uint8 [B,H,N,bs,d],
+    sf4 uint8 [B,H,N,d,bs/16] (group scales of channel c over slots 16g..16g+15).
+    """
+    x = vp.astype(F32)
+    s, inv = outer_scale(amax_c)
+    y = (x * inv[:, :, None, None, :]).astype(F32)
+    q8 = e4m3_code(y)
+    yt = np.swapaxes(y, 3, 4)                        # [B,H,N,d,bs]
+    q4t, sf4 = fp4_groups(yt)
+    return dict(s=s, q8=q8, q4=np.swapaxes(q4t, 3, 4).copy(), sf4=sf4)
+
+
+def dequant_qk(qd, precision: int) -> np.ndarray:
+    """fp64 [B,H,N,bs,d] values of a quantised Q or K copy (8 or 4 bits)."""
+    s = qd["s"].astype(np.float64)[..., None, None]
+    if precision == 8:
+        return s * e4m3_decode(qd["q8"])
+    return s * fp4_dequant(qd["q4"], qd["sf4"])
+
+
+def dequant_v(vd, precision: int) -> np.ndarray:
+    s = vd["s"].astype(np.float64)[:, :, None, None, :]
+    if precision == 8:
+        return s * e4m3_decode(vd["q8"])
+    vt = fp4_dequant(np.swapaxes(vd["q4"], 3, 4), vd["sf4"])
+    return s * np.swapaxes(vt, 3, 4)
+
+
+# ----------------------------------------------------------------------------------------
+# Draft maps and ranking ([DA2] Abstract: low-resolution draft attention map from avg- and
+# max-pooled Q/K estimates block importance; a shared ranking gives high precision, low
+# precision or skip under budgets. [DA1] Abstract / [NEWS] step 2: the draft map is the
+# attention of the pooled queries over the pooled keys.)
+# ----------------------------------------------------------------------------------------
+def draft_scores(qavg, kavg, qmax, kmax, counts, sm_scale, mass_correction=True):
+    """Block-importance score fp64 [B, H, N(query block), N(key block)].
+
+    Each map is a row softmax over key blocks of sm_scale * <pooled q_i, pooled k_j>
+    plus ln(c_j) (c_j valid tokens of key block j, so a map estimates the attention MASS
+    of block j rather than that of one average token). score = (P_avg + P_max) / 2.
+    """
+    lc = np.log(counts.astype(np.float64)) if mass_correction else np.zeros(len(counts))
+
+    def one(qp, kp):
+        lg = sm_scale * np.einsum("bhid,bhjd->bhij", qp.astype(np.float64),
+                                  kp.astype(np.float64)) + lc[None, None, None, :]
+        lg = lg - lg.max(axis=-1, keepdims=True)
+        e = np.exp(lg)
+        return e / e.sum(axis=-1, keepdims=True)
+
+    return 0.5 * (one(qavg, kavg) + one(qmax, kmax))
+
+
+def rank(scores, n8: int, n4: int):
+    """Shared ranking of each row: order (score desc, block index asc); the first n8 blocks
+    are FP8, the next n4 FP4, the rest skipped.
+
+    Returns tags uint8 [..., N, N] (0 skip, 1 FP4, 2 FP8), list8 int [..., N, n8] and
+    list4 int [..., N, n4], each list in ascending block index.
+    """
+    sc = np.asarray(scores)
+    lead = sc.shape[:-1]
+    N = sc.shape[-1]
+    flat = sc.reshape(-1, N)
+    j = np.arange(N)
+    tags = np.zeros(flat.shape, dtype=np.uint8)
+    l8 = np.zeros((flat.shape[0], n8), dtype=np.int64)
+    l4 = np.zeros((flat.shape[0], n4), dtype=np.int64)
+    for r in range(flat.shape[0]):
+        order = np.lexsort((j, -flat[r]))
+        tags[r, order[:n8]] = TAG_FP8
+        tags[r, order[n8:n8 + n4]] = TAG_FP4
+        l8[r] = np.sort(order[:n8])
+        l4[r] = np.sort(order[n8:n8 + n4])
+    return (tags.reshape(lead + (N,)), l8.reshape(lead + (n8,)), l4.reshape(lead + (n4,)))
+
+
+# ----------------------------------------------------------------------------------------
+# P quantisation inside the attention ([DA2] Abstract: both matmuls of a block run at its
+# precision). p = exp(S - m) <= 1 with m the running row max.
+# ----------------------------------------------------------------------------------------
+def quant_p(p: np.ndarray, precision: int) -> np.ndarray:
+    """Quantised probabilities (fp64). FP8: E4M3(448 p)/448. FP4: y = 448 p, groups of 16
+    consecutive keys, sigma = E4M3(amax16/6), value sigma*E2M1(y/sigma)/448."""
+    y = p * E4M3_MAX
+    if precision == 8:
+        return e4m3_round(y) / E4M3_MAX
+    sh = y.shape
+    yg = y.reshape(sh[:-1] + (sh[-1] // 16, 16))
+    sig = e4m3_round(np.abs(yg).max(axis=-1) / E2M1_MAX)
+    safe = np.where(sig > 0, sig, 1.0)
+    z = np.where(sig[..., None] > 0, e2m1_round(yg / safe[..., None]) * sig[..., None], 0.0)
+    return z.reshape(sh) / E4M3_MAX
+
+
+# ----------------------------------------------------------------------------------------
+# Mixed-precision block-sparse attention ([DA2] Abstract: one kernel with precision-
+# specific phases that share data movement, softmax statistics and output accumulation)
+# ----------------------------------------------------------------------------------------
+@dataclass
+class Operands:
+    """fp64 operand values per precision: q8/q4/k8/k4/v8/v4 [B,H,N,bs,d]."""
+    q: dict
+    k: dict
+    v: dict
+
+
+def operands_quantised(qd, kd, vd) -> Operands:
+    return Operands({8: dequant_qk(qd, 8), 4: dequant_qk(qd, 4)},
+                    {8: dequant_qk(kd, 8), 4: dequant_qk(kd, 4)},
+                    {8: dequant_v(vd, 8), 4: dequant_v(vd, 4)})
+
+
+def operands_exact(qp, kp, vp) -> Operands:
+    q, k, v = (x.astype(np.float64) for x in (qp, kp, vp))
+    return Operands({8: q, 4: q}, {8: k, 4: k}, {8: v, 4: v})
+
+
+def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
+              return_parts=False):
+    """Block-sparse attention with one online softmax over both phases.
+
+    For each (b, h, query block i): the FP8 phase visits list8[i] in ascending block index,
+    then the FP4 phase visits list4[i]; each visited block j updates the running row max
+    m, rescales the running sum l and accumulator by exp(m_old - m_new), adds
+    sum(exp(S - m_new)) to l (unquantised) and adds P~ V to the accumulator, with P~ the
+    block's quantised probabilities taken against the running max. Padded key slots are
+    masked (-inf); skipped blocks contribute nothing. Output O = acc / l, fp64
+    [B, H, N, bs, d]; rows with no kept block are 0.
+
+    With return_parts, also returns per (b,h,i) lists of (j, alpha_j, sum p~, sum p~ v)
+    for the error decomposition.
+    """
+    B, H, N, bs, d = ops.q[8].shape
+    out = np.zeros((B, H, N, bs, d))
+    parts = {} if return_parts else None
+    for b in range(B):
+        for h in range(H):
+            for i in range(N):
+                m = np.full(bs, -np.inf)
+                l = np.zeros(bs)
+                acc = np.zeros((bs, d))
+                rec = []
+                for prec, lst in ((8, list8[b, h, i]), (4, list4[b, h, i])):
+                    qi = ops.q[prec][b, h, i]
+                    for j in lst:
+                        S = sm_scale * (qi @ ops.k[prec][b, h, j].T)
+                        S[:, ~valid[j]] = -np.inf
+                        m_new = np.maximum(m, S.max(axis=1))
+                        fin = np.isfinite(m_new)
+                        alpha = np.where(np.isfinite(m), np.exp(m - np.where(fin, m_new, 0.0)), 0.0)
+                        p = np.exp(S - np.where(fin, m_new, 0.0)[:, None])
+                        p[~np.isfinite(S)] = 0.0
+                        pq = quant_p(p, prec) if quantise_p else p
+                        pv = pq @ ops.v[prec][b, h, j]
+                        l = alpha * l + p.sum(axis=1)
+                        acc = alpha[:, None] * acc + pv
+                        if return_parts:
+                            for r in rec:
+                                r[1] *= alpha
+                            rec.append([j, np.ones(bs), pq.sum(axis=1), pv])
+                        m = m_new
+                safe = np.where(l > 0, l, 1.0)
+                out[b, h, i] = np.where(l[:, None] > 0, acc / safe[:, None], 0.0)
+                if return_parts:
+                    parts[(b, h, i)] = (rec, l)
+    return (out, parts) if return_parts else out
+
+
+def dense_attention(q, k, v, sm_scale, key_mask=None):
+    """Textbook softmax attention in fp64 on [B,H,T,d] (key_mask [..., Tq, Tk] bool keeps)."""
+    S = sm_scale * np.einsum("bhqd,bhkd->bhqk", q.astype(np.float64), k.astype(np.float64))
+    if key_mask is not None:
+        S = np.where(key_mask, S, -np.inf)
+    S = S - S.max(axis=-1, keepdims=True)
+    P = np.exp(S)
+    P = P / P.sum(axis=-1, keepdims=True)
+    return np.einsum("bhqk,bhkd->bhqd", P, v.astype(np.float64))
+
+
+# ----------------------------------------------------------------------------------------
+# Error decomposition ([DA2] Abstract: the analysis separates the sparsification error
+# from an attention-weighted quantisation error). The formula is not printed on the pages:
+# parity unpinned. Reading: per query row, with O dense, O_S the exact attention over the
+# kept blocks, O~ the mixed result,
+#   E_sp = ||O_S - O|| = m_skip ||o_skip - O_S||   (m_skip: softmax mass of skipped blocks)
+#   E_q  = sum_b w_b ||o~_b - o_b|| + sum_b |w~_b - w_b| ||o~_b||
+# where w_b / o_b are block b's share of the kept mass and its block-normalised output,
+# and w~_b / o~_b the same quantities from the mixed computation (O~ = sum_b w~_b o~_b).
+# Then ||O~ - O|| <= E_sp + E_q.
+# ----------------------------------------------------------------------------------------
+def error_decomposition(q, k, v, valid, list8, list4, ops_q: Operands, sm_scale, g: Geometry):
+    """Per-row (E_tot, E_sp, E_q, m_skip) arrays [B,H,N,bs] plus (O, O_S, O~)."""
+    qp, kp, vp = (permute(x, g).astype(np.float64) for x in (q, k, v))
+    ops_x = operands_exact(qp, kp, vp)
+    B, H, N, bs, d = qp.shape
+    kept = np.zeros((B, H, N, N), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            for i in range(N):
+                kept[b, h, i, list8[b, h, i]] = True
+                kept[b, h, i, list4[b, h, i]] = True
+    all8 = np.broadcast_to(np.arange(N), (B, H, N, N))
+    none = np.zeros((B, H, N, 0), dtype=np.int64)
+    O = attention(ops_x, valid, all8, none, sm_scale, quantise_p=False)
+    OS, parts_x = attention(ops_x, valid, list8, list4, sm_scale, quantise_p=False,
+                            return_parts=True)
+    Ot, parts_q = attention(ops_q, valid, list8, list4, sm_scale, quantise_p=True,
+                            return_parts=True)
+    E_tot = np.linalg.norm(Ot - O, axis=-1)
+    E_sp = np.linalg.norm(OS - O, axis=-1)
+    E_q = np.zeros((B, H, N, bs))
+    m_skip = np.zeros((B, H, N, bs))
+    for key, (rec_x, l_x) in parts_x.items():
+        rec_q, l_q = parts_q[key]
+        b, h, i = key
+        for (jx, ax, sx, pvx), (jq, aq, sq, pvq) in zip(rec_x, rec_q):
+            assert jx == jq
+            w = ax * sx / np.where(l_x > 0, l_x, 1.0)
+            o = pvx / np.where(sx > 0, sx, 1.0)[:, None]
+            wt = aq * sq / np.where(l_q > 0, l_q, 1.0)
+            ot = pvq / np.where(sq > 0, sq, 1.0)[:, None]
+            E_q[b, h, i] += w * np.linalg.norm(ot - o, axis=-1) + \
+                np.abs(wt - w) * np.linalg.norm(ot, axis=-1)
+    # skipped mass from the dense softmax
+    for b in range(B):
+        for h in range(H):
+            for i in range(N):
+                S = sm_scale * np.einsum("rd,jsd->rjs", qp[b, h, i], kp[b, h])
+                S[:, ~valid] = -np.inf
+                S = S - S.max(axis=(1, 2), keepdims=True)
+                P = np.exp(S)
+                tot = P.sum(axis=(1, 2))
+                skip = P[:, ~kept[b, h, i]].sum(axis=(1, 2))
+                m_skip[b, h, i] = skip / tot
+    return dict(E_tot=E_tot, E_sp=E_sp, E_q=E_q, m_skip=m_skip, O=O, OS=OS, Ot=Ot)
+
+
+# ----------------------------------------------------------------------------------------
+# The whole path
+# ----------------------------------------------------------------------------------------
+def _np(x):
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().cpu().float().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, dtype=F32)
+
+
+def prepare(w, q, k, v):
+    """Pooling, permutation and operand quantisation for inputs [B,H,T,d] (bf16 values)."""
+    g = geometry(w)
+    q, k, v = _np(q), _np(k), _np(v)
+    valid = block_valid(g)
+    qp, kp, vp = permute(q, g), permute(k, g), permute(v, g)
+    qavg, qmax = pool(qp, valid)
+    kavg, kmax = pool(kp, valid)
+    vamax = v_channel_amax(v)
+    return dict(g=g, valid=valid, counts=valid.sum(1), qp=qp, kp=kp, vp=vp,
+                qavg=qavg, qmax=qmax, kavg=kavg, kmax=kmax, vamax=vamax,
+                Q=quantise_qk(qp, valid), K=quantise_qk(kp, valid), V=quantise_v(vp, vamax))
+
+
+def draft_select(prep, mass_correction=True):
+    g = prep["g"]
+    sc = draft_scores(prep["qavg"], prep["kavg"], prep["qmax"], prep["kmax"],
+                      prep["counts"], g.sm_scale, mass_correction)
+    tags, l8, l4 = rank(sc, g.n8, g.n4)
+    return dict(scores=sc, tags=tags, list8=l8, list4=l4)
+
+
+def run(w, q, k, v, quantised=True, lists=None):
+    """Whole hot path. Returns dict with every intermediate and `out` fp64 [B,H,T,d].
+
+    `lists` = (list8, list4) overrides the oracle's own selection (used to compare the
+    attention step on the CUDA path's selection when rankings differ at near-ties).
+    """
+    prep = prepare(w, q, k, v)
+    g = prep["g"]
+    sel = draft_select(prep)
+    l8, l4 = (sel["list8"], sel["list4"]) if lists is None else lists
+    if quantised:
+        ops = operands_quantised(prep["Q"], prep["K"], prep["V"])
+    else:
+        ops = operands_exact(prep["qp"], prep["kp"], prep["vp"])
+    o = attention(ops, prep["valid"], l8, l4, g.sm_scale, quantise_p=quantised)
+    return dict(prep=prep, sel=sel, out_blocks=o, out=inverse_permute(o, g))
