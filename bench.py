@@ -1,0 +1,370 @@
+"""Benchmark of the DraftAttention2 hot path (prepare + draft_select + attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan720] [--impl ours|reference]
+
+One step = one whole attention call on one synthetic Wan2.1-14B-like 720p layer (B=1,
+H=40, d=128, 21x45x80 = 75 600 tokens, 8x16 windows, FP8 10% / FP4 30% / skip 60%),
+inputs resident in HBM. Timed with CUDA events on the launching stream, L2 flushed
+between steps, max over ranks. Under torchrun every rank runs its own replica (weak
+scaling; the path has no exchange step). Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from sparse_mixed_precision_b200.synth import WORKLOADS, generate  # noqa: E402
+
+METRIC = "dense-equivalent TFLOP/s of one DraftAttention2 attention call (75.6k tokens)"
+UNIT = "TFLOP/s"
+KERNELS_PER_STEP = 4      # k_vamax, k_prepare, k_draft_select, attention
+
+
+def dense_flops(w) -> float:
+    return 4.0 * w.B * w.H * float(w.T) ** 2 * w.d
+
+
+def executed_flops(w):
+    """(FP8, FP4) tensor FLOPs actually executed: kept block pairs x 4 bs^2 d."""
+    import math as _m
+    ny, nx = _m.ceil(w.Hf / w.ph), _m.ceil(w.Wf / w.pw)
+    N = w.F * ny * nx
+    bs = w.ph * w.pw
+    n8 = (w.pct_fp8 * N + 50) // 100
+    nk = ((w.pct_fp8 + w.pct_fp4) * N + 50) // 100
+    rows = w.B * w.H * N
+    per = 4.0 * bs * bs * w.d
+    return rows * n8 * per, rows * (nk - n8) * per
+
+
+def prep_bytes(w) -> float:
+    """Algorithmic HBM bytes of the preparation stage (reads once, writes once)."""
+    import math as _m
+    ny, nx = _m.ceil(w.Hf / w.ph), _m.ceil(w.Wf / w.pw)
+    N = w.F * ny * nx
+    bs = w.ph * w.pw
+    BH = w.B * w.H
+    Tp = N * bs
+    kv4 = max(bs, 64)
+    rd = 3 * BH * w.T * w.d * 2
+    wr = BH * Tp * w.d * 3 + BH * Tp * w.d // 2 * 2 + BH * N * w.d * kv4 // 2 \
+        + BH * N * (w.d // 64) * 512 * 2 + BH * N * (kv4 // 64) * 512 + 4 * BH * N * w.d * 4
+    return float(rd + wr)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.lines = index, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------
+# CPU oracle timing (reported baseline; also the reference arm)
+# ------------------------------------------------------------------------------------------
+def oracle_sample(w, q, k, v, n_blocks: int):
+    """Times the oracle on one head: the whole preparation and selection, and the
+    attention of `n_blocks` query blocks; returns (seconds per call extrapolated to all
+    heads and query blocks, description)."""
+    import numpy as np
+    import oracle as O
+    from sparse_mixed_precision_b200.synth import scaled
+    wh = scaled(w, B=1, H=1)
+    qh, kh, vh = (x[:1, :1].cpu() for x in (q, k, v))
+    t0 = time.perf_counter()
+    P = O.prepare(wh, qh, kh, vh)
+    sel = O.draft_select(P)
+    t1 = time.perf_counter()
+    g = P["g"]
+    ops = O.operands_quantised(P["Q"], P["K"], P["V"])
+    blocks = [(0, 0, i) for i in np.linspace(0, g.N - 1, n_blocks).astype(int)]
+    t2 = time.perf_counter()
+    O.attention(ops, P["valid"], sel["list8"], sel["list4"], g.sm_scale, True, blocks=blocks)
+    t3 = time.perf_counter()
+    per_head = (t1 - t0) + (t3 - t2) * g.N / len(blocks)
+    sec = per_head * w.B * w.H
+    desc = (f"oracle on head (0,0): prepare+select {t1 - t0:.2f} s, attention of {len(blocks)}"
+            f" of {g.N} query blocks {t3 - t2:.2f} s; extrapolated x{g.N / len(blocks):.1f}"
+            f" blocks and x{w.B * w.H} heads")
+    return sec, desc
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # pragma: no cover
+        return 1
+
+
+def run_reference(args, w, ws_size, rank):
+    if rank != 0:
+        return
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    q, k, v = generate(w, device=gen_dev)
+    per_step = []
+    desc = ""
+    for s in range(args.warmup + args.steps):
+        sec, desc = oracle_sample(w, q, k, v, args.ref_blocks)
+        if s >= args.warmup:
+            per_step.append(sec)
+    sec = statistics.mean(per_step)
+    value = dense_flops(w) / sec / 1e12
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, args):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} d={w.d} {w.F}x{w.Hf}x{w.Wf} tokens"
+                        f" ({w.T}), window {w.ph}x{w.pw}, FP8 {w.pct_fp8}% / FP4 {w.pct_fp4}%"
+                        f" / skip {100 - w.pct_fp8 - w.pct_fp4}%",
+            "tokens": w.T, "batch": w.B, "heads": w.H, "head_dim": w.d,
+            "l2": "flushed between steps (512 MiB write); inputs 774 MB per tensor",
+            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="wan720", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-blocks", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+    world, rank, local = dist_setup()
+
+    if args.impl == "reference":
+        run_reference(args, w, None, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import sparse_mixed_precision_b200 as da2
+    dev = torch.device("cuda", local)
+    q, k, v = generate(w, device=dev, seed=w.seed + rank)
+    cfg = da2.config(w)
+    views = da2.workspace_views(cfg)
+    ws = torch.empty(views["total"], dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        da2.prepare(cfg, q, k, v, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        da2.draft_select(cfg, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        da2.attention(cfg, ws, out, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert da2.get_error(cfg, ws) == 0
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            flush.zero_()
+            step(events[s])
+        torch.cuda.synchronize()
+    barrier(world)
+    stage = {"prepare": [], "draft_select": [], "attention": []}
+    total = []
+    for ev in events:
+        a, b, c, d = (ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
+                      ev[2].elapsed_time(ev[3]), ev[0].elapsed_time(ev[3]))
+        stage["prepare"].append(a)
+        stage["draft_select"].append(b)
+        stage["attention"].append(c)
+        total.append(d)
+    ms_local = sum(total) / len(total)
+    ms = max_over_ranks(ms_local, world)
+    assert da2.get_error(cfg, ws) == 0
+    value = dense_flops(w) * world / (ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel (attention): precision-weighted tensor bound
+    peaks, src = load_peaks()
+    bf16 = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    p8, p4 = 2.0 * bf16, 4.0 * bf16          # nominal dense ratios fp8 : fp4 : bf16 = 2 : 4 : 1
+    f8, f4 = executed_flops(w)
+    attn_ms = statistics.mean(stage["attention"])
+    t_roof_attn = (f8 / (p8 * 1e12) + f4 / (p4 * 1e12)) * 1e3
+    achieved = (f8 + f4) / (attn_ms * 1e-3) / 1e12
+    peak_eff = (f8 + f4) / (t_roof_attn * 1e-3) / 1e12
+    prep_ms = statistics.mean(stage["prepare"])
+    pb = prep_bytes(w)
+    traffic_path = os.path.join(ROOT, "profiles", "traffic.json")
+    traffic = None
+    if os.path.exists(traffic_path):
+        traffic = json.load(open(traffic_path)).get("attention_bytes_per_launch")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3/e2m1 MMA, f32 accumulate", "data": "synthetic (seeded smooth field + noise + sinks)",
+        "config": config_dict(w, args),
+        "stages_ms": {k_: statistics.mean(v_) for k_, v_ in stage.items()},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff, "unit": "TFLOP/s",
+                     "frac": t_roof_attn / attn_ms, "traffic": traffic,
+                     "note": f"attention kernel; peak = precision-weighted ({f8:.3e} FP8 + {f4:.3e} FP4 FLOP"
+                             f" at {p8:.0f} / {p4:.0f} TFLOP/s = 2x / 4x {src} sustained bf16)"},
+        "prepare_hbm": {"achieved_gbs": pb / (prep_ms * 1e-3) / 1e9, "peak_gbs": peaks["hbm_gbs"],
+                        "frac": pb / (prep_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "step_roofline_frac": (t_roof_attn + pb / (peaks["hbm_gbs"] * 1e9) * 1e3) / ms,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    if not args.no_e2e:
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        da2.forward_host(cfg, qh, kh, vh, oh, q, k, v, out, ws, stream)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(2, min(args.steps, 5))
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            da2.forward_host(cfg, qh, kh, vh, oh, q, k, v, out, ws, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        nbytes = q.numel() * q.element_size()
+        line["e2e"] = {"value": dense_flops(w) * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                       "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * nbytes,
+                       "d2h_bytes_per_step": nbytes}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec, desc = oracle_sample(w, q, k, v, args.ref_blocks)
+        line["cpu_baseline"] = {"value": dense_flops(w) / sec / 1e12, "unit": UNIT,
+                                "cores": blas_threads(), "kind": "oracle", "sample": desc,
+                                "ms_per_call": sec * 1e3}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

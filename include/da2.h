@@ -1,0 +1,167 @@
+/*
+ * da2.h -- C ABI of the DraftAttention2 hot path on NVIDIA B200 (sm_100a).
+ *
+ * Low-resolution-guided, block-sparse, mixed-precision self-attention over
+ * spatiotemporal video-DiT tokens:
+ *
+ *   da2_prepare       fused operand preparation: per-frame 2D average- and max-pooled
+ *                     draft Q/K, window-contiguous token permutation, FP8-E4M3 and
+ *                     4-bit (E2M1, one E4M3 scale per 16 elements) copies of Q/K/V.
+ *   da2_draft_select  low-resolution draft attention maps (avg- and max-pooled) combined
+ *                     into a block-importance score, and the shared per-(head, query
+ *                     block) ranking into FP8 / FP4 / skip under the budgets.
+ *   da2_attention     one attention kernel with an FP8 phase and an FP4 phase that share
+ *                     the online-softmax running max / sum and the fp32 accumulator; its
+ *                     epilogue writes bf16 output back in the original token order.
+ *
+ * Sources: "DraftAttention2: Fast Video Diffusion with Low-Resolution-Guided Mixed-
+ * Precision Attention" (arXiv 2609.32628), Abstract -- pooled draft Q/K, shared ranking
+ * into higher / lower precision / skip under budgets, fused operand preparation, one
+ * attention kernel with precision-specific phases sharing data movement, softmax
+ * statistics and output accumulation. "DraftAttention: Fast Video Diffusion via
+ * Low-Resolution Attention Guidance" (arXiv 2505.14708), Abstract -- per-frame
+ * downsampling into draft Q/K, reorder before and restore after the sparse attention.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Inputs q, k, v and the output are bf16 [B, H, T, d], d contiguous, with frame-major
+ *    token order t = f*Hf*Wf + y*Wf + x.
+ *  - Window (ph, pw) tiles each frame; edge windows are padded. Blocks n = f*ny*nx +
+ *    (y/ph)*nx + (x/pw), slot s = (y%ph)*pw + (x%pw), ny = ceil(Hf/ph), nx = ceil(Wf/pw),
+ *    N = F*ny*nx blocks of bs = ph*pw slots; padded slots hold zeros and padded keys are
+ *    masked out of the attention.
+ *  - Budgets: n8 = floor((pct_fp8*N + 50)/100) FP8 KV blocks and n4 = floor(((pct_fp8 +
+ *    pct_fp4)*N + 50)/100) - n8 FP4 KV blocks per query block; the rest are skipped.
+ *  - Memory ownership: the caller allocates q, k, v, out and the workspace (device memory,
+ *    size from da2_workspace_size); the library allocates nothing and keeps no state.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream) except the ones
+ *    documented as synchronising. Argument errors are returned before anything is
+ *    enqueued; a failed launch returns DA2_ERR_CUDA (see cudaGetLastError for detail).
+ *  - Supported: d in {64, 128}; any window with bs = ph*pw in {32, 64, 128}; N <= 4096;
+ *    0 <= pct_fp8, pct_fp4 and pct_fp8 + pct_fp4 <= 100. Tensor pointers must be 16-byte
+ *    aligned and the workspace 256-byte aligned (DA2_ERR_ALIGNMENT otherwise).
+ */
+#ifndef DA2_H
+#define DA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* One attention call's shape, window and budgets. */
+typedef struct da2_config {
+  int B, H, d;          /* batch, heads, head dim (64 or 128) */
+  int F, Hf, Wf;        /* latent frames, token rows and token columns per frame */
+  int ph, pw;           /* pooling window rows x columns; block size bs = ph*pw */
+  int pct_fp8, pct_fp4; /* percent of KV blocks kept at FP8 / FP4; the rest is skipped */
+  float sm_scale;       /* softmax scale; 0 selects 1/sqrt(d) */
+  int flags;            /* DA2_FLAG_* bits */
+} da2_config;
+
+enum {
+  /* da2_draft_select also writes its fp32 block-importance scores to the workspace
+     (scores region, [B*H][N][N]); the workspace then grows by 4*B*H*N*N bytes. */
+  DA2_FLAG_EXPORT_SCORES = 1,
+  /* Drop the ln(valid tokens) term of the draft logits (the maps then rank by average
+     token affinity instead of block mass). */
+  DA2_FLAG_NO_MASS_CORRECTION = 2
+};
+
+typedef enum da2_status {
+  DA2_OK = 0,
+  DA2_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, budgets out of range */
+  DA2_ERR_UNSUPPORTED = 2,  /* d or bs outside the supported set */
+  DA2_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+  DA2_ERR_WORKSPACE = 4,    /* ws_bytes smaller than da2_workspace_size */
+  DA2_ERR_CUDA = 5,         /* a CUDA call or launch failed */
+  DA2_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out (device error word set) */
+} da2_status;
+
+/* Byte offsets of the workspace regions (from the workspace base) and the geometry.
+   Tile layouts (all per (b*H + h) then per block, each block tile contiguous):
+     q8, k8   E4M3 [BH][N][tile8_qk]: bs rows (tokens) x d bytes in the tensor-core
+              K-major core-matrix layout: byte (r, c) at (r/8)*(8*d) + (c/16)*128 +
+              (r%8)*16 + c%16.
+     q4, k4   E2M1 [BH][N][tile4_qk]: bs rows x d/2 bytes, element c in byte c/2 (even
+              c in the low nibble), byte (r, b) at (r/8)*(4*d) + (b/16)*128 + (r%8)*16 +
+              b%16.
+     v8       E4M3 transposed [BH][N][tile8_v]: d rows (channels) x bs bytes (slots):
+              byte (c, s) at (c/8)*(8*bs) + (s/16)*128 + (c%8)*16 + s%16.
+     v4       E2M1 transposed [BH][N][tile4_v]: d rows x kv4/2 bytes, kv4 = max(bs, 64)
+              (slots >= bs are zero codes): byte (c, b) at (c/8)*(4*kv4) + (b/16)*128 +
+              (c%8)*16 + b%16.
+     sfq4, sfk4  E4M3 group scales of q4/k4, [BH][N][sf_qk]: d/64 atoms of 512 bytes;
+              atom kb holds rows 0..127 (rows >= bs zero) x 4 scales (channel groups
+              4kb..4kb+3): byte (r, j) at kb*512 + (r%32)*16 + (r/32)*4 + j.
+     sfv4     E4M3 group scales of v4, [BH][N][sf_v]: kv4/64 atoms; rows = channels
+              (rows >= d zero), scales = slot groups: byte (c, j) at kb*512 + (c%32)*16 +
+              (c/32)*4 + j for slot group 4kb + j (groups past bs are zero).
+     sq, sk   fp32 [BH][N]   dequantisation scale of a Q / K block (block amax / 448).
+     sv       fp32 [BH][d]   dequantisation scale of a V channel (channel amax / 448).
+     vamax    fp32 [BH][d]   V channel amax (written by da2_prepare).
+     qavg, qmax, kavg, kmax  fp32 [BH][N][d] pooled draft Q / K.
+     tags     u8 [BH][N][N]  0 skip, 1 FP4, 2 FP8 for (query block, KV block).
+     list8    i16 [BH][N][n8s], list4 i16 [BH][N][n4s]: kept KV blocks per query block
+              in ascending block order (n8s = max(n8,1), n4s = max(n4,1)).
+     scores   fp32 [BH][N][N] (only with DA2_FLAG_EXPORT_SCORES, else size 0).
+     err      u32 device error word (0 = no error). */
+typedef struct da2_views {
+  int N, bs, T, Tp, ny, nx, n8, n4, kv4;
+  size_t tile8_qk, tile4_qk, tile8_v, tile4_v, sf_qk, sf_v;
+  size_t q8, k8, v8, q4, k4, v4, sfq4, sfk4, sfv4;
+  size_t sq, sk, sv, vamax, qavg, qmax, kavg, kmax;
+  size_t tags, list8, list4, scores, err, total;
+} da2_views;
+
+/* Workspace bytes needed for `cfg` (host only, no CUDA call). */
+da2_status da2_workspace_size(const da2_config* cfg, size_t* bytes);
+
+/* Geometry and region offsets for `cfg` (host only, no CUDA call). */
+da2_status da2_workspace_views(const da2_config* cfg, da2_views* views);
+
+/* Operand preparation. q, k, v: device bf16 [B,H,T,d]; ws: device workspace of at least
+   da2_workspace_size bytes. Writes every operand, scale and pooled region of ws and
+   clears its error word. Asynchronous on `stream`. */
+da2_status da2_prepare(const da2_config* cfg, const void* q, const void* k, const void* v,
+                       void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Draft maps and ranking on a prepared workspace: writes tags, list8, list4 (and scores
+   with DA2_FLAG_EXPORT_SCORES). Asynchronous on `stream`. */
+da2_status da2_draft_select(const da2_config* cfg, void* ws, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/* Mixed-precision block-sparse attention on a prepared and selected workspace. out:
+   device bf16 [B,H,T,d] (every element is written). Bounded device waits that run out
+   set the workspace error word (read it with da2_get_error). Asynchronous. */
+da2_status da2_attention(const da2_config* cfg, void* ws, size_t ws_bytes, void* out,
+                         cudaStream_t stream);
+
+/* da2_prepare, da2_draft_select and da2_attention in order on one stream. */
+da2_status da2_forward(const da2_config* cfg, const void* q, const void* k, const void* v,
+                       void* out, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Host-buffer variant of da2_forward: copies q, k, v (host, bf16 [B,H,T,d]; pinned
+   memory gives asynchronous copies) into the caller's device staging buffers dq, dk, dv,
+   runs the three stages and copies the result from dout back to out_host, all on
+   `stream`. Synchronises `stream` before returning so out_host is ready. */
+da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const void* k_host,
+                            const void* v_host, void* out_host, void* dq, void* dk,
+                            void* dv, void* dout, void* ws, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/* Reads the workspace's device error word into *word and clears it (synchronises
+   `stream`). Returns DA2_ERR_TIMEOUT if the word was non-zero. */
+da2_status da2_get_error(void* ws, size_t ws_bytes, const da2_config* cfg,
+                         cudaStream_t stream, uint32_t* word);
+
+/* Static string naming a status. */
+const char* da2_status_string(da2_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DA2_H */

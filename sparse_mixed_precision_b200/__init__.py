@@ -1,0 +1,154 @@
+"""Python binding of libda2 (the DraftAttention2 hot path on B200, sm_100a).
+
+Argument marshalling only: every step of the path runs in the CUDA library. The names
+follow the C ABI in include/da2.h. Tensors are torch tensors (device memory and streams
+come from PyTorch); the library itself allocates nothing.
+
+    cfg = config(workload)                      # da2_config from a synth.Workload
+    ws  = torch.empty(workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    prepare(cfg, q, k, v, ws); draft_select(cfg, ws); attention(cfg, ws, out)
+
+The extension must be built first (`python -m sparse_mixed_precision_b200.build` or
+`__graft_entry__.build()`); there is no fallback when it is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libda2.so")
+
+FLAG_EXPORT_SCORES = 1
+FLAG_NO_MASS_CORRECTION = 2
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned pointer",
+          4: "workspace too small", 5: "CUDA error", 6: "device error word set"}
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "d", "F", "Hf", "Wf", "ph", "pw",
+                                             "pct_fp8", "pct_fp4")] + \
+               [("sm_scale", ctypes.c_float), ("flags", ctypes.c_int)]
+
+
+_VIEW_INTS = ("N", "bs", "T", "Tp", "ny", "nx", "n8", "n4", "kv4")
+_VIEW_SIZES = ("tile8_qk", "tile4_qk", "tile8_v", "tile4_v", "sf_qk", "sf_v",
+               "q8", "k8", "v8", "q4", "k4", "v4", "sfq4", "sfk4", "sfv4",
+               "sq", "sk", "sv", "vamax", "qavg", "qmax", "kavg", "kmax",
+               "tags", "list8", "list4", "scores", "err", "total")
+
+
+class Views(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in _VIEW_INTS] + [(n, ctypes.c_size_t) for n in _VIEW_SIZES]
+
+
+class DA2Error(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libda2.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libda2.so not built ({LIB_PATH}); run sparse_mixed_precision_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, cp = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Config)
+        sigs = {
+            "da2_workspace_size": [cp, ctypes.POINTER(ctypes.c_size_t)],
+            "da2_workspace_views": [cp, ctypes.POINTER(Views)],
+            "da2_prepare": [cp, vp, vp, vp, vp, sz, vp],
+            "da2_draft_select": [cp, vp, sz, vp],
+            "da2_attention": [cp, vp, sz, vp, vp],
+            "da2_forward": [cp, vp, vp, vp, vp, vp, sz, vp],
+            "da2_forward_host": [cp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "da2_get_error": [vp, sz, cp, vp, ctypes.POINTER(ctypes.c_uint32)],
+        }
+        for name, args in sigs.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.da2_status_string.argtypes = [ctypes.c_int]
+        L.da2_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+EXPORTED = ("da2_workspace_size", "da2_workspace_views", "da2_prepare", "da2_draft_select",
+            "da2_attention", "da2_forward", "da2_forward_host", "da2_get_error",
+            "da2_status_string")
+
+
+def config(w, flags: int = 0, sm_scale: float = 0.0) -> Config:
+    """da2_config of a synth.Workload (or any object with the same fields)."""
+    return Config(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, w.pct_fp8, w.pct_fp4,
+                  float(sm_scale), int(flags))
+
+
+def _check(fn, st):
+    if st != 0:
+        raise DA2Error(fn, st)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(cfg: Config) -> int:
+    n = ctypes.c_size_t()
+    _check("da2_workspace_size", lib().da2_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def workspace_views(cfg: Config) -> dict:
+    v = Views()
+    _check("da2_workspace_views", lib().da2_workspace_views(ctypes.byref(cfg), ctypes.byref(v)))
+    return {n: getattr(v, n) for n in _VIEW_INTS + _VIEW_SIZES}
+
+
+def prepare(cfg, q, k, v, ws, stream=None):
+    _check("da2_prepare", lib().da2_prepare(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def draft_select(cfg, ws, stream=None):
+    _check("da2_draft_select", lib().da2_draft_select(ctypes.byref(cfg), _ptr(ws), ws.numel(),
+                                                      _stream(stream)))
+
+
+def attention(cfg, ws, out, stream=None):
+    _check("da2_attention", lib().da2_attention(ctypes.byref(cfg), _ptr(ws), ws.numel(),
+                                                _ptr(out), _stream(stream)))
+
+
+def forward(cfg, q, k, v, out, ws, stream=None):
+    _check("da2_forward", lib().da2_forward(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def forward_host(cfg, q_host, k_host, v_host, out_host, dq, dk, dv, dout, ws, stream=None):
+    _check("da2_forward_host", lib().da2_forward_host(
+        ctypes.byref(cfg), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(out_host),
+        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dout), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def get_error(cfg, ws, stream=None) -> int:
+    """Reads and clears the workspace's device error word (synchronises the stream)."""
+    word = ctypes.c_uint32()
+    st = lib().da2_get_error(_ptr(ws), ws.numel(), ctypes.byref(cfg), _stream(stream),
+                             ctypes.byref(word))
+    if st not in (0, 6):
+        raise DA2Error("da2_get_error", st)
+    return word.value

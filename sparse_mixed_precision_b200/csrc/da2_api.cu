@@ -1,0 +1,242 @@
+// C ABI of the da2 library: argument checks, workspace layout and stage launches.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace da2 {
+cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
+                           const void* v, cudaStream_t st);
+cudaError_t launch_draft_select(const Geo& g, const Ws& w, cudaStream_t st);
+cudaError_t launch_attention(const Geo& g, const Ws& w, void* out, cudaStream_t st);
+}  // namespace da2
+
+using namespace da2;
+
+namespace {
+
+constexpr int kMaxBlocks = 4096;
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+da2_status check_config(const da2_config* c) {
+  if (!c) return DA2_ERR_INVALID_ARG;
+  if (c->B <= 0 || c->H <= 0 || c->F <= 0 || c->Hf <= 0 || c->Wf <= 0 || c->ph <= 0 || c->pw <= 0)
+    return DA2_ERR_INVALID_ARG;
+  if (c->pct_fp8 < 0 || c->pct_fp4 < 0 || c->pct_fp8 + c->pct_fp4 > 100) return DA2_ERR_INVALID_ARG;
+  if (!(c->sm_scale >= 0.0f) || std::isinf(c->sm_scale)) return DA2_ERR_INVALID_ARG;
+  if (c->d != 64 && c->d != 128) return DA2_ERR_UNSUPPORTED;
+  const long bs = (long)c->ph * c->pw;
+  if (bs != 32 && bs != 64 && bs != 128) return DA2_ERR_UNSUPPORTED;
+  const long ny = (c->Hf + c->ph - 1) / c->ph, nx = (c->Wf + c->pw - 1) / c->pw;
+  const long N = (long)c->F * ny * nx;
+  if (N > kMaxBlocks) return DA2_ERR_UNSUPPORTED;
+  if ((long)c->B * c->H * N * N > (1L << 40)) return DA2_ERR_UNSUPPORTED;
+  return DA2_OK;
+}
+
+void fill_views(const da2_config* c, da2_views* v) {
+  std::memset(v, 0, sizeof(*v));
+  v->ny = (c->Hf + c->ph - 1) / c->ph;
+  v->nx = (c->Wf + c->pw - 1) / c->pw;
+  v->N = c->F * v->ny * v->nx;
+  v->bs = c->ph * c->pw;
+  v->T = c->F * c->Hf * c->Wf;
+  v->Tp = v->N * v->bs;
+  v->n8 = (c->pct_fp8 * v->N + 50) / 100;
+  v->n4 = ((c->pct_fp8 + c->pct_fp4) * v->N + 50) / 100 - v->n8;
+  v->kv4 = v->bs < 64 ? 64 : v->bs;
+  const size_t d = c->d, bs = v->bs, N = v->N, BH = (size_t)c->B * c->H;
+  v->tile8_qk = bs * d;
+  v->tile4_qk = bs * d / 2;
+  v->tile8_v = d * bs;
+  v->tile4_v = d * v->kv4 / 2;
+  v->sf_qk = (d / 64) * 512;
+  v->sf_v = (v->kv4 / 64) * 512;
+  const size_t n8s = v->n8 > 0 ? v->n8 : 1, n4s = v->n4 > 0 ? v->n4 : 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + bytes); return o; };
+  v->q8 = take(BH * N * v->tile8_qk);
+  v->k8 = take(BH * N * v->tile8_qk);
+  v->v8 = take(BH * N * v->tile8_v);
+  v->q4 = take(BH * N * v->tile4_qk);
+  v->k4 = take(BH * N * v->tile4_qk);
+  v->v4 = take(BH * N * v->tile4_v);
+  v->sfq4 = take(BH * N * v->sf_qk);
+  v->sfk4 = take(BH * N * v->sf_qk);
+  v->sfv4 = take(BH * N * v->sf_v);
+  v->sq = take(BH * N * 4);
+  v->sk = take(BH * N * 4);
+  v->sv = take(BH * d * 4);
+  v->vamax = take(BH * d * 4);
+  v->qavg = take(BH * N * d * 4);
+  v->qmax = take(BH * N * d * 4);
+  v->kavg = take(BH * N * d * 4);
+  v->kmax = take(BH * N * d * 4);
+  v->tags = take(BH * N * N);
+  v->list8 = take(BH * N * n8s * 2);
+  v->list4 = take(BH * N * n4s * 2);
+  v->scores = take((c->flags & DA2_FLAG_EXPORT_SCORES) ? BH * N * N * 4 : 0);
+  v->err = take(4);
+  v->total = off;
+}
+
+Geo make_geo(const da2_config* c, const da2_views& v) {
+  Geo g;
+  g.B = c->B; g.H = c->H; g.d = c->d; g.F = c->F; g.Hf = c->Hf; g.Wf = c->Wf;
+  g.ph = c->ph; g.pw = c->pw; g.ny = v.ny; g.nx = v.nx; g.N = v.N; g.bs = v.bs;
+  g.T = v.T; g.Tp = v.Tp; g.n8 = v.n8; g.n4 = v.n4; g.kv4 = v.kv4;
+  g.sm_scale = c->sm_scale > 0.0f ? c->sm_scale : 1.0f / std::sqrt((float)c->d);
+  g.flags = c->flags;
+  return g;
+}
+
+Ws make_ws(void* base, const da2_views& v) {
+  uint8_t* b = static_cast<uint8_t*>(base);
+  Ws w;
+  w.q8 = b + v.q8; w.k8 = b + v.k8; w.v8 = b + v.v8;
+  w.q4 = b + v.q4; w.k4 = b + v.k4; w.v4 = b + v.v4;
+  w.sfq4 = b + v.sfq4; w.sfk4 = b + v.sfk4; w.sfv4 = b + v.sfv4;
+  w.sq = reinterpret_cast<float*>(b + v.sq);
+  w.sk = reinterpret_cast<float*>(b + v.sk);
+  w.sv = reinterpret_cast<float*>(b + v.sv);
+  w.vamax = reinterpret_cast<float*>(b + v.vamax);
+  w.qavg = reinterpret_cast<float*>(b + v.qavg);
+  w.qmax = reinterpret_cast<float*>(b + v.qmax);
+  w.kavg = reinterpret_cast<float*>(b + v.kavg);
+  w.kmax = reinterpret_cast<float*>(b + v.kmax);
+  w.scores = reinterpret_cast<float*>(b + v.scores);
+  w.tags = b + v.tags;
+  w.list8 = reinterpret_cast<int16_t*>(b + v.list8);
+  w.list4 = reinterpret_cast<int16_t*>(b + v.list4);
+  w.err = reinterpret_cast<uint32_t*>(b + v.err);
+  w.tile8_qk = v.tile8_qk; w.tile4_qk = v.tile4_qk; w.tile8_v = v.tile8_v; w.tile4_v = v.tile4_v;
+  w.sf_qk = v.sf_qk; w.sf_v = v.sf_v;
+  w.n8s = v.n8 > 0 ? v.n8 : 1;
+  w.n4s = v.n4 > 0 ? v.n4 : 1;
+  return w;
+}
+
+// Common checks for the stage calls; fills views / geo / ws on success.
+da2_status setup(const da2_config* cfg, void* ws, size_t ws_bytes, da2_views* v, Geo* g, Ws* w) {
+  da2_status s = check_config(cfg);
+  if (s != DA2_OK) return s;
+  if (!ws) return DA2_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DA2_ERR_ALIGNMENT;
+  fill_views(cfg, v);
+  if (ws_bytes < v->total) return DA2_ERR_WORKSPACE;
+  *g = make_geo(cfg, *v);
+  *w = make_ws(ws, *v);
+  return DA2_OK;
+}
+
+da2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DA2_OK : DA2_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+da2_status da2_workspace_size(const da2_config* cfg, size_t* bytes) {
+  const da2_status s = check_config(cfg);
+  if (s != DA2_OK) return s;
+  if (!bytes) return DA2_ERR_INVALID_ARG;
+  da2_views v;
+  fill_views(cfg, &v);
+  *bytes = v.total;
+  return DA2_OK;
+}
+
+da2_status da2_workspace_views(const da2_config* cfg, da2_views* views) {
+  const da2_status s = check_config(cfg);
+  if (s != DA2_OK) return s;
+  if (!views) return DA2_ERR_INVALID_ARG;
+  fill_views(cfg, views);
+  return DA2_OK;
+}
+
+da2_status da2_prepare(const da2_config* cfg, const void* q, const void* k, const void* v,
+                       void* ws, size_t ws_bytes, cudaStream_t stream) {
+  da2_views vw; Geo g; Ws w;
+  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
+  if (s != DA2_OK) return s;
+  if (!q || !k || !v) return DA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return DA2_ERR_ALIGNMENT;
+  return cuda_status(launch_prepare(g, w, q, k, v, stream));
+}
+
+da2_status da2_draft_select(const da2_config* cfg, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  da2_views vw; Geo g; Ws w;
+  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
+  if (s != DA2_OK) return s;
+  return cuda_status(launch_draft_select(g, w, stream));
+}
+
+da2_status da2_attention(const da2_config* cfg, void* ws, size_t ws_bytes, void* out,
+                         cudaStream_t stream) {
+  da2_views vw; Geo g; Ws w;
+  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
+  if (s != DA2_OK) return s;
+  if (!out) return DA2_ERR_INVALID_ARG;
+  if (!aligned16(out)) return DA2_ERR_ALIGNMENT;
+  return cuda_status(launch_attention(g, w, out, stream));
+}
+
+da2_status da2_forward(const da2_config* cfg, const void* q, const void* k, const void* v,
+                       void* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  da2_status s = da2_prepare(cfg, q, k, v, ws, ws_bytes, stream);
+  if (s != DA2_OK) return s;
+  s = da2_draft_select(cfg, ws, ws_bytes, stream);
+  if (s != DA2_OK) return s;
+  return da2_attention(cfg, ws, ws_bytes, out, stream);
+}
+
+da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const void* k_host,
+                            const void* v_host, void* out_host, void* dq, void* dk, void* dv,
+                            void* dout, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const da2_status s0 = check_config(cfg);
+  if (s0 != DA2_OK) return s0;
+  if (!q_host || !k_host || !v_host || !out_host || !dq || !dk || !dv || !dout)
+    return DA2_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)cfg->B * cfg->H * cfg->F * cfg->Hf * cfg->Wf * cfg->d * 2;
+  cudaError_t e = cudaMemcpyAsync(dq, q_host, bytes, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, bytes, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, bytes, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  const da2_status s = da2_forward(cfg, dq, dk, dv, dout, ws, ws_bytes, stream);
+  if (s != DA2_OK) return s;
+  e = cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  return cuda_status(e);
+}
+
+da2_status da2_get_error(void* ws, size_t ws_bytes, const da2_config* cfg, cudaStream_t stream,
+                         uint32_t* word) {
+  da2_views vw; Geo g; Ws w;
+  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
+  if (s != DA2_OK) return s;
+  if (!word) return DA2_ERR_INVALID_ARG;
+  uint32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, w.err, 4, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(w.err, 0, 4, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  *word = h;
+  return h ? DA2_ERR_TIMEOUT : DA2_OK;
+}
+
+const char* da2_status_string(da2_status s) {
+  switch (s) {
+    case DA2_OK: return "ok";
+    case DA2_ERR_INVALID_ARG: return "invalid argument";
+    case DA2_ERR_UNSUPPORTED: return "unsupported shape";
+    case DA2_ERR_ALIGNMENT: return "misaligned pointer";
+    case DA2_ERR_WORKSPACE: return "workspace too small";
+    case DA2_ERR_CUDA: return "CUDA error";
+    case DA2_ERR_TIMEOUT: return "device error word set (bounded wait ran out or bad index)";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,237 @@
+// Operand preparation (HBM-bound): V channel amax pre-pass and the fused prepare kernel.
+//
+// "DraftAttention2: Fast Video Diffusion with Low-Resolution-Guided Mixed-Precision
+// Attention", Abstract: draft queries/keys are spatial 2D average- and max-pooled, and a
+// fused operand-preparation step feeds the mixed-precision attention kernel.
+// "DraftAttention: Fast Video Diffusion via Low-Resolution Attention Guidance", Abstract:
+// per-frame downsampling; tokens are reordered so that each pooled region is contiguous.
+//
+// One CTA prepares one (b, h, block) of one tensor: it stages the window's tokens (bf16,
+// 128-bit loads, padded slots zero) in shared memory once, then writes the pooled draft
+// vectors (Q, K), the E4M3 copy and the E2M1 copy with its E4M3 group scales in the tile
+// layouts the attention kernel loads directly (see include/da2.h).
+#include "common.cuh"
+
+namespace da2 {
+
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(uint4 u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// ---- K0: amax of V over all tokens, per (b, h, channel) ----
+// grid (chunks, B*H); vamax must be zero on entry (non-negative floats compare as uints).
+template <int D>
+__global__ void __launch_bounds__(256) k_vamax(const __nv_bfloat16* __restrict__ v,
+                                               float* __restrict__ vamax, int T, int chunk) {
+  constexpr int VPR = D / 8;          // 16-byte vectors per token
+  constexpr int RSTEP = 256 / VPR;    // tokens per sweep
+  __shared__ float red[RSTEP][D + 1];
+  const int bh = blockIdx.y;
+  const int t0 = blockIdx.x * chunk, t1 = min(T, t0 + chunk);
+  const int cv = threadIdx.x % VPR, tr = threadIdx.x / VPR;
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+  const __nv_bfloat16* base = v + (size_t)bh * T * D;
+  for (int t = t0 + tr; t < t1; t += RSTEP) {
+    float f[8];
+    bf16x8_to_f32(ld_stream_u4(base + (size_t)t * D + cv * 8), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(f[i]));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[tr][cv * 8 + i] = m[i];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += 256) {
+    float a = 0.0f;
+    for (int r = 0; r < RSTEP; ++r) a = fmaxf(a, red[r][c]);
+    atomicMax(reinterpret_cast<unsigned int*>(vamax + (size_t)bh * D + c), __float_as_uint(a));
+  }
+}
+
+// ---- K1: fused preparation of one (b, h, block) of Q, K (pool + quantise) or V ----
+// grid (N, B*H, 3); blockIdx.z: 0 = Q, 1 = K, 2 = V.
+template <int D>
+__global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat16* __restrict__ q,
+                                                 const __nv_bfloat16* __restrict__ k,
+                                                 const __nv_bfloat16* __restrict__ v) {
+  constexpr int RS = D + 8;           // smem row stride (bf16), padded against bank conflicts
+  constexpr int VPR = D / 8;
+  extern __shared__ __align__(16) uint8_t smem[];
+  __nv_bfloat16* X = reinterpret_cast<__nv_bfloat16*>(smem);
+  const int bs = g.bs;
+  uint8_t* sfbuf = smem + (size_t)bs * RS * 2;             // up to 1 KB of group scales
+  float* red = reinterpret_cast<float*>(sfbuf + 1024);      // 8 floats of reduction scratch
+
+  const int n = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const int tid = threadIdx.x;
+  const __nv_bfloat16* src = which == 0 ? q : (which == 1 ? k : v);
+  const int fpf = g.ny * g.nx;
+  const int f = n / fpf, rem = n - f * fpf, by = rem / g.nx, bx = rem - by * g.nx;
+  const int y0 = by * g.ph, x0 = bx * g.pw;
+  const int hv = min(g.ph, g.Hf - y0), wv = min(g.pw, g.Wf - x0);
+
+  // stage the window (padded slots zero)
+  const __nv_bfloat16* sbase = src + (size_t)bh * g.T * D;
+  for (int u = tid; u < bs * VPR; u += 256) {
+    const int s = u / VPR, cv = u - s * VPR;
+    const int wy = s / g.pw, wx = s - wy * g.pw;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (wy < hv && wx < wv) {
+      const size_t t = (size_t)f * g.Hf * g.Wf + (size_t)(y0 + wy) * g.Wf + (x0 + wx);
+      val = ld_stream_u4(sbase + t * D + cv * 8);
+    }
+    *reinterpret_cast<uint4*>(X + s * RS + cv * 8) = val;
+  }
+  const int sfbytes = which < 2 ? (int)w.sf_qk : (int)w.sf_v;
+  for (int i = tid; i < sfbytes / 4; i += 256) reinterpret_cast<uint32_t*>(sfbuf)[i] = 0u;
+  __syncthreads();
+
+  if (which < 2) {
+    // ---- draft pooling: fp32 running sum in slot order, then IEEE divide; exact max ----
+    float* avg_out = (which == 0 ? w.qavg : w.kavg) + ((size_t)bh * g.N + n) * D;
+    float* max_out = (which == 0 ? w.qmax : w.kmax) + ((size_t)bh * g.N + n) * D;
+    if (tid < 2 * D) {
+      const int c = tid % D;
+      const bool do_sum = tid < D;
+      float acc = do_sum ? 0.0f : -INFINITY;
+      for (int s = 0; s < bs; ++s) {
+        const int wy = s / g.pw, wx = s - wy * g.pw;
+        if (wy < hv && wx < wv) {
+          const float x = __bfloat162float(X[s * RS + c]);
+          acc = do_sum ? __fadd_rn(acc, x) : fmaxf(acc, x);
+        }
+      }
+      if (do_sum) avg_out[c] = __fdiv_rn(acc, (float)(hv * wv));
+      else max_out[c] = acc;
+    }
+    // ---- block amax -> outer scale ----
+    float am = 0.0f;
+    for (int u = tid; u < bs * VPR; u += 256) {
+      const int s = u / VPR, cv = u - s * VPR;
+      float fv[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(X + s * RS + cv * 8), fv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(fv[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    if ((tid & 31) == 0) red[tid >> 5] = am;
+    __syncthreads();
+    am = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) am = fmaxf(am, red[i]);
+    const float inv = am > 0.0f ? __fdiv_rn(kE4M3Max, am) : 1.0f;
+    if (tid == 0) (which == 0 ? w.sq : w.sk)[(size_t)bh * g.N + n] = am > 0.0f ? __fdiv_rn(am, kE4M3Max) : 1.0f;
+
+    // ---- E4M3 and E2M1 copies, one 16-channel chunk of one token per step ----
+    uint8_t* t8 = (which == 0 ? w.q8 : w.k8) + ((size_t)bh * g.N + n) * w.tile8_qk;
+    uint8_t* t4 = (which == 0 ? w.q4 : w.k4) + ((size_t)bh * g.N + n) * w.tile4_qk;
+    constexpr int KC = D / 16;
+    for (int u = tid; u < bs * KC; u += 256) {
+      const int rg = u / (8 * KC), within = u - rg * 8 * KC;
+      const int kc = within >> 3, rr = within & 7;
+      const int r = rg * 8 + rr;
+      float y[16];
+      float xf[16];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(X + r * RS + kc * 16), xf);
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(X + r * RS + kc * 16 + 8), xf + 8);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(xf[i], inv);
+      uint32_t p8[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        p8[i] = (uint32_t)f32x2_to_e4m3x2(y[4 * i], y[4 * i + 1]) |
+                ((uint32_t)f32x2_to_e4m3x2(y[4 * i + 2], y[4 * i + 3]) << 16);
+      *reinterpret_cast<uint4*>(t8 + (size_t)u * 16) = make_uint4(p8[0], p8[1], p8[2], p8[3]);
+      uint32_t p4[2];
+      const uint8_t sc = quant_fp4_group16(y, p4);
+      *reinterpret_cast<uint2*>(t4 + kmajor_off(r, kc * 8, D / 2)) = make_uint2(p4[0], p4[1]);
+      sfbuf[sf_off(kc >> 2, r, kc & 3)] = sc;
+    }
+    __syncthreads();
+    uint8_t* sfo = (which == 0 ? w.sfq4 : w.sfk4) + ((size_t)bh * g.N + n) * w.sf_qk;
+    for (int i = tid; i < sfbytes / 16; i += 256)
+      reinterpret_cast<uint4*>(sfo)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
+  } else {
+    // ---- V: per-channel outer scale from the amax pre-pass; tiles are channel-major ----
+    const float* am = w.vamax + (size_t)bh * D;
+    if (n == 0)
+      for (int c = tid; c < D; c += 256)
+        w.sv[(size_t)bh * D + c] = am[c] > 0.0f ? __fdiv_rn(am[c], kE4M3Max) : 1.0f;
+    uint8_t* t8 = w.v8 + ((size_t)bh * g.N + n) * w.tile8_v;
+    uint8_t* t4 = w.v4 + ((size_t)bh * g.N + n) * w.tile4_v;
+    const int SC = bs / 16, SC4 = g.kv4 / 16;
+    for (int u = tid; u < D * SC4; u += 256) {
+      const int cg = u / (8 * SC4), within = u - cg * 8 * SC4;
+      const int sc = within >> 3, cc = within & 7;
+      const int c = cg * 8 + cc;
+      const float a = am[c];
+      const float inv = a > 0.0f ? __fdiv_rn(kE4M3Max, a) : 1.0f;
+      float y[16];
+      if (sc < SC) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(__bfloat162float(X[(sc * 16 + i) * RS + c]), inv);
+        uint32_t p8[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          p8[i] = (uint32_t)f32x2_to_e4m3x2(y[4 * i], y[4 * i + 1]) |
+                  ((uint32_t)f32x2_to_e4m3x2(y[4 * i + 2], y[4 * i + 3]) << 16);
+        *reinterpret_cast<uint4*>(t8 + kmajor_off(c, sc * 16, bs)) = make_uint4(p8[0], p8[1], p8[2], p8[3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = 0.0f;
+      }
+      uint32_t p4[2];
+      const uint8_t s4 = quant_fp4_group16(y, p4);
+      *reinterpret_cast<uint2*>(t4 + kmajor_off(c, sc * 8, g.kv4 / 2)) = make_uint2(p4[0], p4[1]);
+      sfbuf[sf_off(sc >> 2, c, sc & 3)] = s4;
+    }
+    __syncthreads();
+    uint8_t* sfo = w.sfv4 + ((size_t)bh * g.N + n) * w.sf_v;
+    for (int i = tid; i < sfbytes / 16; i += 256)
+      reinterpret_cast<uint4*>(sfo)[i] = reinterpret_cast<const uint4*>(sfbuf)[i];
+  }
+}
+
+size_t prepare_smem_bytes(const Geo& g) {
+  return (size_t)g.bs * (g.d + 8) * 2 + 1024 + 64;
+}
+
+cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
+                           const void* v, cudaStream_t st) {
+  const int BH = g.B * g.H;
+  cudaError_t e = cudaMemsetAsync(w.vamax, 0, sizeof(float) * BH * g.d, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(w.err, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  const int chunk = 2048;
+  dim3 g0((g.T + chunk - 1) / chunk, BH);
+  const size_t smem = prepare_smem_bytes(g);
+  dim3 g1(g.N, BH, 3);
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  if (g.d == 128) {
+    k_vamax<128><<<g0, 256, 0, st>>>(vb, w.vamax, g.T, chunk);
+    k_prepare<128><<<g1, 256, smem, st>>>(g, w, qb, kb, vb);
+  } else {
+    k_vamax<64><<<g0, 256, 0, st>>>(vb, w.vamax, g.T, chunk);
+    k_prepare<64><<<g1, 256, smem, st>>>(g, w, qb, kb, vb);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace da2

@@ -1,0 +1,73 @@
+"""The C-ABI library loads and exports every symbol include/*.h declares; host-only calls
+(workspace size / views, argument validation) behave as documented. No compute calls."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import sparse_mixed_precision_b200 as da2
+from sparse_mixed_precision_b200.synth import WORKLOADS, scaled
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names |= set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(da2_[a-z_0-9]+)\s*\(",
+                                src, re.M))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert {"da2_prepare", "da2_draft_select", "da2_attention"} <= names
+    L = da2.lib()
+    for n in sorted(names):
+        assert hasattr(L, n), n
+    assert set(da2.EXPORTED) >= names - set()  # the binding wraps every declared call
+
+
+def test_workspace_views_consistent():
+    for name in ("tiny", "wan480", "wan720", "hunyuan720"):
+        w = WORKLOADS[name]
+        cfg = da2.config(w)
+        v = da2.workspace_views(cfg)
+        assert v["total"] == da2.workspace_size(cfg)
+        import oracle as O
+        g = O.geometry(w)
+        assert (v["N"], v["bs"], v["T"], v["Tp"], v["n8"], v["n4"]) == (g.N, g.bs, g.T, g.Tp, g.n8, g.n4)
+        offs = sorted((v[k], k) for k in ("q8", "k8", "v8", "q4", "k4", "v4", "sfq4", "sfk4",
+                                           "sfv4", "sq", "sk", "sv", "tags", "list8", "err"))
+        assert all(o % 256 == 0 for o, _ in offs)
+        assert len({o for o, _ in offs}) == len(offs)
+    # exporting scores grows the workspace by 4 B H N^2 (rounded to 256)
+    w = WORKLOADS["tiny"]
+    a = da2.workspace_size(da2.config(w))
+    b = da2.workspace_size(da2.config(w, flags=da2.FLAG_EXPORT_SCORES))
+    assert b - a >= 4 * w.B * w.H * 64 * 64
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(d=96), 2), (dict(ph=3, pw=8), 2), (dict(pct_fp8=60, pct_fp4=50), 1),
+    (dict(pct_fp8=-1), 1), (dict(B=0), 1), (dict(F=200, Hf=90, Wf=160), 2),
+])
+def test_invalid_configs_rejected(change, status):
+    cfg = da2.config(scaled(WORKLOADS["tiny"], **change))
+    n = ctypes.c_size_t()
+    assert da2.lib().da2_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == status
+
+
+def test_stage_calls_reject_bad_pointers_without_touching_the_device():
+    L = da2.lib()
+    cfg = da2.config(WORKLOADS["tiny"])
+    n = da2.workspace_size(cfg)
+    # null workspace / misaligned workspace / too-small workspace: checked on the host
+    assert L.da2_draft_select(ctypes.byref(cfg), None, n, None) == 1
+    assert L.da2_draft_select(ctypes.byref(cfg), ctypes.c_void_p(0x1008), n, None) == 3
+    assert L.da2_draft_select(ctypes.byref(cfg), ctypes.c_void_p(0x100000), n - 1, None) == 4
+    assert L.da2_prepare(ctypes.byref(cfg), None, None, None, ctypes.c_void_p(0x100000), n, None) == 1
+    assert L.da2_status_string(6).startswith(b"device error word")
