@@ -396,7 +396,7 @@ def operands_exact(qp, kp, vp) -> Operands:
 
 
 def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
-              return_parts=False):
+              return_parts=False, blocks=None):
     """Block-sparse attention with one online softmax over both phases.
 
     For each (b, h, query block i): the FP8 phase visits list8[i] in ascending block index,
@@ -408,14 +408,15 @@ def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
     [B, H, N, bs, d]; rows with no kept block are 0.
 
     With return_parts, also returns per (b,h,i) lists of (j, alpha_j, sum p~, sum p~ v)
-    for the error decomposition.
+    for the error decomposition. `blocks`, a list of (b, h, i), restricts the computation
+    to those query blocks (the others stay 0).
     """
     B, H, N, bs, d = ops.q[8].shape
     out = np.zeros((B, H, N, bs, d))
     parts = {} if return_parts else None
-    for b in range(B):
-        for h in range(H):
-            for i in range(N):
+    todo = blocks if blocks is not None else [(b, h, i) for b in range(B) for h in range(H)
+                                              for i in range(N)]
+    for b, h, i in todo:
                 m = np.full(bs, -np.inf)
                 l = np.zeros(bs)
                 acc = np.zeros((bs, d))

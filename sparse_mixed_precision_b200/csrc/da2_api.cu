@@ -8,7 +8,7 @@ namespace da2 {
 cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
                            const void* v, cudaStream_t st);
 cudaError_t launch_draft_select(const Geo& g, const Ws& w, cudaStream_t st);
-cudaError_t launch_attention(const Geo& g, const Ws& w, void* out, cudaStream_t st);
+cudaError_t launch_attention_tc(const Geo& g, const Ws& w, void* out, cudaStream_t st);
 }  // namespace da2
 
 using namespace da2;
@@ -180,7 +180,7 @@ da2_status da2_attention(const da2_config* cfg, void* ws, size_t ws_bytes, void*
   if (s != DA2_OK) return s;
   if (!out) return DA2_ERR_INVALID_ARG;
   if (!aligned16(out)) return DA2_ERR_ALIGNMENT;
-  return cuda_status(launch_attention(g, w, out, stream));
+  return cuda_status(launch_attention_tc(g, w, out, stream));
 }
 
 da2_status da2_forward(const da2_config* cfg, const void* q, const void* k, const void* v,
