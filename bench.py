@@ -236,10 +236,15 @@ def main():
     ap.add_argument("--workload", default="wan720", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-blocks", type=int, default=8)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (small cases for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
+    if args.heads > 0:
+        from sparse_mixed_precision_b200.synth import scaled
+        w = scaled(w, H=args.heads)
     world, rank, local = dist_setup()
 
     if args.impl == "reference":

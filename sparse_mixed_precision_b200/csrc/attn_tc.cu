@@ -18,11 +18,13 @@
 //   O += P~ V_j'             same MMA kind as the block, accumulating into the one O.
 // Epilogue: out = O s_v / (448 l) in bf16, written to the tokens' original positions.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work items in head-major
+// Warp roles (320 threads, one CTA per SM, persistent over work items in head-major
 // order so that one head's K/V stay in L2):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r) and the epilogue
-//   warp 4     MMA issue (one thread) and TMEM allocation
-//   warp 5     producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
+//   warps 0-7  softmax + epilogue: warps w and w+4 own query rows 32(w%4)..+31 (TMEM
+//              lane quarter w%4) and split the key columns of S / P and the output
+//              columns of O between them
+//   warp 8     MMA issue (one thread) and TMEM allocation
+//   warp 9     producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
 // Every mbarrier wait is bounded; a wait that runs out sets the workspace error word and
 // the kernel carries on to a clean exit.
 #include "common.cuh"
@@ -31,11 +33,29 @@
 namespace da2 {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kMmaWarp = 4;
-constexpr int kLoadWarp = 5;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;   // warps 0-7
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
 constexpr int kStages = 4;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2_448 = 8.807354922057604f;     // log2(448)
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // TMEM columns (512 allocated)
 constexpr uint32_t kColO = 0, kColS = 128, kColSFQ = 384, kColSFK = 392, kColSFP = 408,
@@ -49,7 +69,9 @@ constexpr uint32_t kStage0 = kSFQ + 1024;
 constexpr uint32_t kStK = 0, kStV = 16384, kStSFK = 32768, kStSFV = 33792, kStageBytes = 34816;
 constexpr uint32_t kP0 = kStage0 + kStages * kStageBytes;
 constexpr uint32_t kPData = 0, kPSF = 16384, kPBytes = 17408;
-constexpr uint32_t kBar = kP0 + 2 * kPBytes;
+constexpr uint32_t kRed = kP0 + 2 * kPBytes;      // row-max exchange [2 parity][2 half][128]
+constexpr uint32_t kLx = kRed + 2 * 2 * 128 * 4;   // row-sum exchange [2 half][128]
+constexpr uint32_t kBar = kLx + 2 * 128 * 4;
 constexpr uint32_t kSmemBytes = kBar + 256;
 
 struct Bars {
@@ -85,12 +107,139 @@ __device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint32_t* 
   }
 }
 
+// Named barrier for the two softmax warps that share a TMEM lane quarter (64 threads).
+__device__ __forceinline__ void pair_sync(int quarter) {
+  asm volatile("bar.sync %0, 64;" ::"r"(quarter + 1) : "memory");
+}
+
 __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, int& wv) {
   const int fpf = g.ny * g.nx;
   const int rem = n % fpf, by = rem / g.nx, bx = rem - by * g.nx;
   hv = min(g.ph, g.Hf - by * g.ph);
   wv = min(g.pw, g.Wf - bx * g.pw);
   return hv * wv;
+}
+
+// One KV block of one query row half (softmax warps). S half-row from TMEM -> group
+// maxima -> row max shared with the partner warp -> alpha -> one fused loop computing
+// p448 = 2^(S c + log2 448 - m_new), the row sum and the quantised P bytes (E4M3, or E2M1
+// with an E4M3 scale per 16 keys) stored straight into the P tile -> O rescale by alpha
+// in TMEM when the max moved (after the previous P V has finished) -> P ready.
+template <int D, int BS, bool FP8>
+__device__ __forceinline__ void softmax_block(const Geo& g, const Ws& w, Bars* bars, uint8_t* sm, uint32_t tmem,
+                                              uint32_t lane_base, float* red, int half, int quarter, int r,
+                                              int j, int bh, float sq, uint32_t gblk, int t, float& m, float& l) {
+  constexpr int HB = BS / 2, HD = D / 2, NG = HB / 16;
+  constexpr int KV4 = BS < 64 ? 64 : BS;
+  const float c = sq * w.sk[(size_t)bh * g.N + j] * g.sm_scale * kLog2e;
+  int hv, wv;
+  const bool edge = block_valid_rows(g, j, hv, wv) < BS;
+  const uint32_t b = gblk & 1, pb = gblk & 1;
+  wait_bar(&bars->s_full[b], (gblk >> 1) & 1, w.err);
+  tc::fence_after_sync();
+  uint32_t sr[HB];
+#pragma unroll
+  for (int c0 = 0; c0 < HB; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColS + b * 128 + half * HB + c0, sr + c0);
+  tc::tmem_wait_ld();
+  tc::fence_before_sync();
+  tc::mbar_arrive(&bars->s_free[b]);
+  float* s = reinterpret_cast<float*>(sr);
+  if (edge) {
+#pragma unroll
+    for (int k = 0; k < HB; ++k) {
+      const int kk = half * HB + k;
+      const int ky = kk / g.pw, kx = kk - ky * g.pw;
+      if (!(ky < hv && kx < wv)) s[k] = -INFINITY;
+    }
+  }
+  // group maxima of the raw dot products (c > 0, so they order like S)
+  float gm[NG];
+#pragma unroll
+  for (int q = 0; q < NG; ++q) {
+    const float* x = s + 16 * q;
+    gm[q] = fmaxf(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8])),
+                  max3(max3(x[9], x[10], x[11]), max3(x[12], x[13], x[14]), x[15]));
+  }
+  float mh = gm[0];
+#pragma unroll
+  for (int q = 1; q < NG; ++q) mh = fmaxf(mh, gm[q]);
+  float* rp = red + (gblk & 1) * 256;
+  rp[half * 128 + r] = mh * c;
+  pair_sync(quarter);
+  const float m_new = fmaxf(m, fmaxf(rp[r], rp[128 + r]));
+  const float alpha = ex2(m - m_new);
+  const float bias = kLog2_448 - m_new;
+  // the P buffer is free once the P V two blocks back has completed
+  if (gblk >= 2) wait_bar(&bars->p_free[pb], ((gblk >> 1) & 1) ^ 1, w.err);
+  uint8_t* pbuf = sm + kP0 + pb * kPBytes;
+  float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (FP8) {
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
+      uint32_t wd[4];
+#pragma unroll
+      for (int e = 0; e < 16; e += 4) {
+        float p[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          p[u] = ex2(fmaf(s[16 * q + e + u], c, bias));
+          sum4[u] += p[u];
+        }
+        wd[e / 4] = (uint32_t)f32x2_to_e4m3x2(p[0], p[1]) | ((uint32_t)f32x2_to_e4m3x2(p[2], p[3]) << 16);
+      }
+      *reinterpret_cast<uint4*>(pbuf + kPData + kmajor_off(r, half * HB + 16 * q, BS)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+    }
+  } else {
+    uint8_t* sfrow = pbuf + kPSF + (r & 31) * 16 + (r >> 5) * 4;
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
+      const int gk = half * HB + 16 * q;                 // first key of the group
+      // group scale from the group max: sigma = E4M3(448 p_max / 6)
+      uint32_t sc = f32_to_e4m3(ex2(fmaf(gm[q], c, bias)) * (1.0f / 6.0f));
+      const float sg = e4m3_to_f32((uint8_t)sc);
+      const float rs = sg > 0.0f ? rcp_approx(sg) : 0.0f;
+      float y[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float p = ex2(fmaf(s[16 * q + e], c, bias));
+        sum4[e & 3] += p;
+        y[e] = p * rs;
+      }
+      const uint2 pk = make_uint2(f32x8_to_e2m1x8(y), f32x8_to_e2m1x8(y + 8));
+      *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, gk / 2, KV4 / 2)) = pk;
+      sfrow[(gk >> 6) * 512 + ((gk >> 4) & 3)] = (uint8_t)sc;
+    }
+    if (KV4 > BS && half == 1) {                           // zero keys past the block (32-token blocks)
+#pragma unroll
+      for (int gk = BS; gk < KV4; gk += 16) {
+        *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, gk / 2, KV4 / 2)) = make_uint2(0u, 0u);
+        sfrow[(gk >> 6) * 512 + ((gk >> 4) & 3)] = 0;
+      }
+    }
+  }
+  l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+  // O rows of this warp's half *= alpha, once the previous P V has landed
+  if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+    const uint32_t gp = gblk - 1;
+    wait_bar(&bars->p_free[gp & 1], (gp >> 1) & 1, w.err);
+    tc::fence_after_sync();
+#pragma unroll
+    for (int h0 = 0; h0 < HD; h0 += 32) {
+      uint32_t orr[32];
+      tc::tmem_ld16(tmem + lane_base + kColO + half * HD + h0, orr);
+      tc::tmem_ld16(tmem + lane_base + kColO + half * HD + h0 + 16, orr + 16);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+      tc::tmem_st16(tmem + lane_base + kColO + half * HD + h0, orr);
+      tc::tmem_st16(tmem + lane_base + kColO + half * HD + h0 + 16, orr + 16);
+    }
+    tc::tmem_wait_st();
+  }
+  m = m_new;
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  tc::mbar_arrive(&bars->p_full[pb]);
 }
 
 template <int D, int BS>
@@ -111,14 +260,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&bars->s_full[b], 1);
-      tc::mbar_init(&bars->s_free[b], 128);
-      tc::mbar_init(&bars->p_full[b], 128);
+      tc::mbar_init(&bars->s_free[b], kSoftmaxThreads);
+      tc::mbar_init(&bars->p_full[b], kSoftmaxThreads);
       tc::mbar_init(&bars->p_free[b], 1);
     }
     tc::mbar_init(&bars->q_full, 1);
     tc::mbar_init(&bars->q_empty, 1);
     tc::mbar_init(&bars->o_full, 1);
-    tc::mbar_init(&bars->o_free, 128);
+    tc::mbar_init(&bars->o_free, kSoftmaxThreads);
     tc::mbar_init(&bars->done, 1);
     tc::fence_mbar_init();
   }
@@ -251,9 +400,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       wait_bar(&bars->done, 0, w.err, false);   // all MMAs retired before TMEM is freed
     }
   } else {
-    // ===================== softmax + epilogue (warps 0-3) =====================
-    const int r = tid;                                   // query row = TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ===================== softmax + epilogue (warps 0-7) =====================
+    // Warps w and w+4 share TMEM lane quarter w%4 (query rows 32(w%4) .. +31); warp
+    // w/4 = h takes key columns [h BS/2, (h+1) BS/2) of S and P and output columns
+    // [h D/2, (h+1) D/2) of O. The row max of each block and the final row sum are
+    // exchanged through shared memory under a named barrier of the pair.
+    constexpr int HB = BS / 2, HD = D / 2;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;                   // query row = TMEM lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    float* red = reinterpret_cast<float*>(sm + kRed);
+    float* lx = reinterpret_cast<float*>(sm + kLx);
     const int fpf = g.ny * g.nx;
     uint32_t gblk = 0, wi = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x, ++wi) {
@@ -267,11 +424,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       if (row_ok) {
         const int f = i / fpf, rem = i - f * fpf, by = rem / g.nx, bx = rem - by * g.nx;
         const size_t t = (size_t)f * g.Hf * g.Wf + (size_t)(by * g.ph + wy) * g.Wf + bx * g.pw + wx;
-        orow = out + ((size_t)bh * g.T + t) * D;
+        orow = out + ((size_t)bh * g.T + t) * D + half * HD;
       }
       if (nb == 0) {
         if (row_ok)
-          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0u, 0u, 0u, 0u);
+          for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0u, 0u, 0u, 0u);
         continue;
       }
       const float sq = w.sq[qi];
@@ -279,140 +436,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       const int16_t* l4 = w.list4 + qi * w.n4s;
       float m = -INFINITY, l = 0.0f;
       for (int t = 0; t < nb; ++t, ++gblk) {
-        const bool fp8 = t < n8;
-        int j = fp8 ? l8[t] : l4[t - n8];
+        int j = t < n8 ? l8[t] : l4[t - n8];
         if (j < 0 || j >= N) j = 0;
-        const float c = sq * w.sk[(size_t)bh * N + j] * g.sm_scale * kLog2e;
-        int hv, wv;
-        const bool edge = block_valid_rows(g, j, hv, wv) < BS;
-        const uint32_t b = gblk & 1, pb = gblk & 1;
-        // ---- S row from TMEM ----
-        wait_bar(&bars->s_full[b], (gblk >> 1) & 1, w.err);
-        tc::fence_after_sync();
-        float s[BS];
-#pragma unroll
-        for (int c0 = 0; c0 < BS; c0 += 16) {
-          uint32_t rr[16];
-          tc::tmem_ld16(tmem + lane_base + kColS + b * 128 + c0, rr);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) s[c0 + e] = __uint_as_float(rr[e]);
-        }
-        tc::fence_before_sync();
-        tc::mbar_arrive(&bars->s_free[b]);
-        // ---- online softmax (log2 domain) ----
-        if (edge) {
-#pragma unroll
-          for (int k = 0; k < BS; ++k) {
-            const int ky = k / g.pw, kx = k - ky * g.pw;
-            if (!(ky < hv && kx < wv)) s[k] = -INFINITY;
-          }
-        }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < BS; ++k) mx = fmaxf(mx, s[k]);
-        const float m_new = fmaxf(m, mx * c);
-        const float alpha = exp2f(m - m_new);
-        float sum = 0.0f;
-#pragma unroll
-        for (int k = 0; k < BS; ++k) {
-          s[k] = exp2f(fmaf(s[k], c, -m_new));
-          sum += s[k];
-        }
-        l = fmaf(l, alpha, sum);
-        // ---- wait for the P buffer (PV two blocks back) and, if the max moved, for the
-        //      previous PV, then rescale this warp's O rows in TMEM ----
-        if (gblk >= 2) wait_bar(&bars->p_free[pb], ((gblk >> 1) & 1) ^ 1, w.err);
-        const bool need = t > 0 && __any_sync(0xffffffffu, alpha != 1.0f);
-        if (need) {
-          const uint32_t gp = gblk - 1;
-          wait_bar(&bars->p_free[gp & 1], (gp >> 1) & 1, w.err);
-          tc::fence_after_sync();
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t rr[16];
-            tc::tmem_ld16(tmem + lane_base + kColO + c0, rr);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-            tc::tmem_st16(tmem + lane_base + kColO + c0, rr);
-          }
-          tc::tmem_wait_st();
-        }
-        m = m_new;
-        // ---- quantise P and write row r of the P tile (K-major core-matrix layout) ----
-        uint8_t* pbuf = sm + kP0 + pb * kPBytes;
-        if (fp8) {
-#pragma unroll
-          for (int c0 = 0; c0 < BS; c0 += 16) {
-            uint32_t wd[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              wd[q] = (uint32_t)f32x2_to_e4m3x2(s[c0 + 4 * q] * kE4M3Max, s[c0 + 4 * q + 1] * kE4M3Max) |
-                      ((uint32_t)f32x2_to_e4m3x2(s[c0 + 4 * q + 2] * kE4M3Max, s[c0 + 4 * q + 3] * kE4M3Max) << 16);
-            *reinterpret_cast<uint4*>(pbuf + kPData + kmajor_off(r, c0, BS)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-          }
-        } else {
-          uint32_t sfw[KV4 / 64];
-#pragma unroll
-          for (int q = 0; q < KV4 / 64; ++q) sfw[q] = 0u;
-#pragma unroll
-          for (int g0 = 0; g0 < KV4; g0 += 16) {
-            uint32_t pk[2] = {0u, 0u};
-            uint32_t sc = 0u;
-            if (g0 < BS) {
-              float y[16];
-              float am = 0.0f;
-#pragma unroll
-              for (int e = 0; e < 16; ++e) am = fmaxf(am, s[g0 + e]);
-              sc = f32_to_e4m3(am * (kE4M3Max / 6.0f));
-              const float sg = e4m3_to_f32((uint8_t)sc);
-              if (sg > 0.0f) {
-                const float rs = kE4M3Max / sg;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) y[e] = s[g0 + e] * rs;
-                pk[0] = f32x8_to_e2m1x8(y);
-                pk[1] = f32x8_to_e2m1x8(y + 8);
-              } else {
-                sc = 0u;
-              }
-            }
-            sfw[g0 / 64] |= sc << (8 * ((g0 / 16) & 3));
-            *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, g0 / 2, KV4 / 2)) = make_uint2(pk[0], pk[1]);
-          }
-#pragma unroll
-          for (int q = 0; q < KV4 / 64; ++q)
-            *reinterpret_cast<uint32_t*>(pbuf + kPSF + q * 512 + (r & 31) * 16 + (r >> 5) * 4) = sfw[q];
-        }
-        tc::fence_proxy_async_smem();
-        tc::fence_before_sync();
-        tc::mbar_arrive(&bars->p_full[pb]);
+        if (t < n8)
+          softmax_block<D, BS, true>(g, w, bars, sm, tmem, lane_base, red, half, quarter, r, j, bh, sq, gblk, t, m, l);
+        else
+          softmax_block<D, BS, false>(g, w, bars, sm, tmem, lane_base, red, half, quarter, r, j, bh, sq, gblk, t, m, l);
       }
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
+      lx[half * 128 + r] = l;
+      pair_sync(quarter);
+      const float lt = lx[r] + lx[128 + r];          // 448 * row sum
       wait_bar(&bars->o_full, wi & 1, w.err);
       tc::fence_after_sync();
-      const float inv = l > 0.0f ? 1.0f / (l * kE4M3Max) : 0.0f;
-      const float* sv = w.sv + (size_t)bh * D;
+      const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
+      const float* sv = w.sv + (size_t)bh * D + half * HD;
+      uint32_t rr[HD];
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t rr[16];
-        tc::tmem_ld16(tmem + lane_base + kColO + c0, rr);
-        tc::tmem_wait_ld();
-        if (row_ok) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float a = __uint_as_float(rr[2 * e]) * __ldg(sv + c0 + 2 * e) * inv;
-            const float bq = __uint_as_float(rr[2 * e + 1]) * __ldg(sv + c0 + 2 * e + 1) * inv;
-            const __nv_bfloat162 h = __floats2bfloat162_rn(a, bq);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          *reinterpret_cast<uint4*>(orow + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(orow + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-      }
+      for (int c0 = 0; c0 < HD; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColO + half * HD + c0, rr + c0);
+      tc::tmem_wait_ld();
       tc::fence_before_sync();
       tc::mbar_arrive(&bars->o_free);
+      if (row_ok) {
+#pragma unroll
+        for (int c0 = 0; c0 < HD; c0 += 8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int cc = c0 + 2 * e;
+            const float a = __uint_as_float(rr[cc]) * __ldg(sv + cc) * inv;
+            const float bq = __uint_as_float(rr[cc + 1]) * __ldg(sv + cc + 1) * inv;
+            const __nv_bfloat162 hh = __floats2bfloat162_rn(a, bq);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&hh);
+          }
+          *reinterpret_cast<uint4*>(orow + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      pair_sync(quarter);                            // lx is reused by the next work item
     }
   }
   tc::fence_before_sync();
