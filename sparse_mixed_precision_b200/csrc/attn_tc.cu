@@ -38,6 +38,7 @@ constexpr int kSoftmaxThreads = 256;   // warps 0-7
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr int kStages = 4;
+constexpr int kPrefetch = 8;   // KV blocks the producer warms in L2 ahead of its copies
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;     // log2(448)
 
@@ -120,8 +121,8 @@ __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, in
   return hv * wv;
 }
 
-// One KV block of one query row half (softmax warps). S half-row from TMEM -> group
-// maxima -> row max shared with the partner warp -> alpha -> one fused loop computing
+// One KV block of one query row half (softmax warps). Both halves of the S row from TMEM
+// (the partner's half only for the row max) -> group maxima -> alpha -> one fused loop computing
 // p448 = 2^(S c + log2 448 - m_new), the row sum and the quantised P bytes (E4M3, or E2M1
 // with an E4M3 scale per 16 keys) stored straight into the P tile -> O rescale by alpha
 // in TMEM when the max moved (after the previous P V has finished) -> P ready.
@@ -287,19 +288,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
     // ===================== producer =====================
     if (lane == 0) {
       uint32_t gblk = 0, wi = 0;
+      auto kv_prefetch = [&](int bh, const int16_t* l8, const int16_t* l4, int t) {
+        const bool fp8 = t < n8;
+        int j = fp8 ? l8[t] : l4[t - n8];
+        if (j < 0 || j >= N) j = 0;
+        const size_t kj = (size_t)bh * N + j;
+        if (fp8) {
+          tc::prefetch_l2(w.k8 + kj * w.tile8_qk, BS * D);
+          tc::prefetch_l2(w.v8 + kj * w.tile8_v, BS * D);
+        } else {
+          tc::prefetch_l2(w.k4 + kj * w.tile4_qk, BS * D / 2);
+          tc::prefetch_l2(w.v4 + kj * w.tile4_v, D * KV4 / 2);
+        }
+      };
       for (int item = blockIdx.x; item < total; item += gridDim.x, ++wi) {
         if (nb == 0) continue;
         const int bh = item / N, i = item - bh * N;
         const size_t qi = (size_t)bh * N + i;
+        const int16_t* l8 = w.list8 + qi * w.n8s;
+        const int16_t* l4 = w.list4 + qi * w.n4s;
+        for (int t = 0; t < kPrefetch && t < nb; ++t) kv_prefetch(bh, l8, l4, t);
         wait_bar(&bars->q_empty, (wi & 1) ^ 1, w.err);
         const uint32_t qbytes = BS * D + BS * D / 2 + (uint32_t)w.sf_qk;
         tc::mbar_arrive_expect_tx(&bars->q_full, qbytes);
         tc::bulk_g2s(sm + kQ8, w.q8 + qi * w.tile8_qk, BS * D, &bars->q_full);
         tc::bulk_g2s(sm + kQ4, w.q4 + qi * w.tile4_qk, BS * D / 2, &bars->q_full);
         tc::bulk_g2s(sm + kSFQ, w.sfq4 + qi * w.sf_qk, (uint32_t)w.sf_qk, &bars->q_full);
-        const int16_t* l8 = w.list8 + qi * w.n8s;
-        const int16_t* l4 = w.list4 + qi * w.n4s;
+        const int nxt = item + gridDim.x;             // warm L2 with the next work item's Q
+        if (nxt < total) {
+          const size_t qn = (size_t)(nxt / N) * N + (nxt % N);
+          tc::prefetch_l2(w.q8 + qn * w.tile8_qk, BS * D);
+          tc::prefetch_l2(w.q4 + qn * w.tile4_qk, BS * D / 2);
+        }
         for (int t = 0; t < nb; ++t, ++gblk) {
+          if (t + kPrefetch < nb) kv_prefetch(bh, l8, l4, t + kPrefetch);
           const bool fp8 = t < n8;
           int j = fp8 ? l8[t] : l4[t - n8];
           if (j < 0 || j >= N) { set_error(w.err, kErrBadIndex); j = 0; }
@@ -386,12 +408,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           tc::mma_commit(&bars->p_free[pb]);
           tc::mma_commit(&bars->kv_empty[s]);
         };
+        // S of the first two blocks, then each P V as soon as its P is ready, followed by
+        // the S two blocks ahead (so a late K/V tile never holds back a P V)
         issue_s(0);
-        for (int t = 1; t < nb; ++t) {
-          issue_s(t);
-          issue_pv(t - 1);
+        if (nb > 1) issue_s(1);
+        for (int t = 0; t < nb; ++t) {
+          issue_pv(t);
+          if (t + 2 < nb) issue_s(t + 2);
         }
-        issue_pv(nb - 1);
         tc::mma_commit(&bars->q_empty);
         tc::mma_commit(&bars->o_full);
         gblk += nb;
