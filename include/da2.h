@@ -78,7 +78,9 @@ typedef enum da2_status {
   DA2_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
   DA2_ERR_WORKSPACE = 4,    /* ws_bytes smaller than da2_workspace_size */
   DA2_ERR_CUDA = 5,         /* a CUDA call or launch failed */
-  DA2_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out (device error word set) */
+  DA2_ERR_TIMEOUT = 6,      /* a kernel's bounded wait ran out (device error word set) */
+  DA2_ERR_SCRATCH_TOO_SMALL = 7 /* da2_forward_noalloc: the configuration's workspace does
+                                   not fit the library's built-in 64 MiB device scratch */
 } da2_status;
 
 /* Byte offsets of the workspace regions (from the workspace base) and the geometry.
@@ -152,6 +154,26 @@ da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const voi
                             const void* v_host, void* out_host, void* dq, void* dk,
                             void* dv, void* dout, void* ws, size_t ws_bytes,
                             cudaStream_t stream);
+
+/* da2_forward without any device allocation, by the library or by the caller.
+   No counterpart in the paper: this serves callers that cannot obtain device memory when
+   they run the attention -- a plug-in inside a host framework that owns all device memory
+   and exposes no allocator, or a serving loop that forbids cudaMalloc after start-up (it
+   can synchronise the device and fail under fragmentation). The caller still passes q,
+   k, v and out (device bf16 [B,H,T,d], 16-byte aligned); the workspace is a fixed 64 MiB
+   device array inside the library, which every GPU that loads the library holds until
+   the process exits. Configurations whose da2_workspace_size exceeds 64 MiB are rejected
+   with DA2_ERR_SCRATCH_TOO_SMALL before anything is enqueued (the tiny workload and
+   single-head 480p / 720p Wan-like layers fit; a full 40-head layer does not). The first call on a
+   device looks up the array's device address (cudaGetSymbolAddress, with that device
+   current); make that first call before any stream capture. Every call on a device shares
+   the one array and leaves its contents behind; the path clears what must start at zero
+   itself. Calls that overlap on the GPU (different streams, or several host threads on
+   one device) race on the array and give wrong results: serialise them. Asynchronous on
+   `stream` like da2_forward. The built-in workspace is not exposed, so its device error
+   word cannot be read with da2_get_error. */
+da2_status da2_forward_noalloc(const da2_config* cfg, const void* q, const void* k,
+                               const void* v, void* out, cudaStream_t stream);
 
 /* Reads the workspace's device error word into *word and clears it (synchronises
    `stream`). Returns DA2_ERR_TIMEOUT if the word was non-zero. */

@@ -23,7 +23,8 @@ FLAG_EXPORT_SCORES = 1
 FLAG_NO_MASS_CORRECTION = 2
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned pointer",
-          4: "workspace too small", 5: "CUDA error", 6: "device error word set"}
+          4: "workspace too small", 5: "CUDA error", 6: "device error word set",
+          7: "workspace larger than the built-in 64 MiB device scratch"}
 
 
 class Config(ctypes.Structure):
@@ -69,6 +70,7 @@ def lib():
             "da2_forward": [cp, vp, vp, vp, vp, vp, sz, vp],
             "da2_forward_host": [cp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "da2_get_error": [vp, sz, cp, vp, ctypes.POINTER(ctypes.c_uint32)],
+            "da2_forward_noalloc": [cp, vp, vp, vp, vp, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -82,7 +84,7 @@ def lib():
 
 EXPORTED = ("da2_workspace_size", "da2_workspace_views", "da2_prepare", "da2_draft_select",
             "da2_attention", "da2_forward", "da2_forward_host", "da2_get_error",
-            "da2_status_string")
+            "da2_status_string", "da2_forward_noalloc")
 
 
 def config(w, flags: int = 0, sm_scale: float = 0.0) -> Config:
@@ -142,6 +144,14 @@ def forward_host(cfg, q_host, k_host, v_host, out_host, dq, dk, dv, dout, ws, st
     _check("da2_forward_host", lib().da2_forward_host(
         ctypes.byref(cfg), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(out_host),
         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dout), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def forward_noalloc(cfg, q, k, v, out, stream=None):
+    """The whole path with the library's built-in 64 MiB device scratch as workspace, for
+    callers that cannot allocate device memory (see da2_forward_noalloc in include/da2.h).
+    Calls on one device must not overlap on the GPU: they share that scratch."""
+    _check("da2_forward_noalloc", lib().da2_forward_noalloc(
+        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _stream(stream)))
 
 
 def get_error(cfg, ws, stream=None) -> int:

@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libda2.so")
-SOURCES = ["da2_api.cu", "prep.cu", "draft.cu", "attn_tc.cu"]
+SOURCES = ["da2_api.cu", "prep.cu", "draft.cu", "attn_tc.cu", "da2_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

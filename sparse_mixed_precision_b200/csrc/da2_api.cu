@@ -235,6 +235,7 @@ const char* da2_status_string(da2_status s) {
     case DA2_ERR_WORKSPACE: return "workspace too small";
     case DA2_ERR_CUDA: return "CUDA error";
     case DA2_ERR_TIMEOUT: return "device error word set (bounded wait ran out or bad index)";
+    case DA2_ERR_SCRATCH_TOO_SMALL: return "workspace larger than the built-in 64 MiB device scratch";
   }
   return "unknown status";
 }
