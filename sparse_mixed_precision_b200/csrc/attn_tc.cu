@@ -18,13 +18,14 @@
 //   O += P~ V_j'             same MMA kind as the block, accumulating into the one O.
 // Epilogue: out = O s_v / (448 l) in bf16, written to the tokens' original positions.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over work items in head-major
+// Warp roles (192 threads, one CTA per SM, persistent over work items in head-major
 // order so that one head's K/V stay in L2):
-//   warps 0-7  softmax + epilogue: warps w and w+4 own query rows 32(w%4)..+31 (TMEM
-//              lane quarter w%4) and split the key columns of S / P and the output
-//              columns of O between them
-//   warp 8     MMA issue (one thread) and TMEM allocation
-//   warp 9     producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
+//   warps 0-3  softmax + epilogue: thread r owns query row r (TMEM lane r), all key
+//              columns of S / P and all output columns of O; one softmax warp per SM
+//              sub-partition, so its short per-block bookkeeping never competes for
+//              issue slots with another warp's exponential loop
+//   warp 4     MMA issue (one thread) and TMEM allocation
+//   warp 5     producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
 // Every mbarrier wait is bounded; a wait that runs out sets the workspace error word and
 // the kernel carries on to a clean exit.
 #include "common.cuh"
@@ -33,10 +34,10 @@
 namespace da2 {
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kSoftmaxThreads = 256;   // warps 0-7
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;   // warps 0-3
+constexpr int kMmaWarp = 4;
+constexpr int kLoadWarp = 5;
 constexpr int kStages = 4;
 constexpr int kPrefetch = 8;   // KV blocks the producer warms in L2 ahead of its copies
 constexpr float kLog2e = 1.4426950408889634f;
@@ -70,9 +71,9 @@ constexpr uint32_t kStage0 = kSFQ + 1024;
 constexpr uint32_t kStK = 0, kStV = 16384, kStSFK = 32768, kStSFV = 33792, kStageBytes = 34816;
 constexpr uint32_t kP0 = kStage0 + kStages * kStageBytes;
 constexpr uint32_t kPData = 0, kPSF = 16384, kPBytes = 17408;
-constexpr uint32_t kRed = kP0 + 2 * kPBytes;      // row-max exchange [2 parity][2 half][128]
-constexpr uint32_t kLx = kRed + 2 * 2 * 128 * 4;   // row-sum exchange [2 half][128]
-constexpr uint32_t kBar = kLx + 2 * 128 * 4;
+constexpr uint32_t kMask = kP0 + 2 * kPBytes;      // 4 slot-validity masks x 4 words
+constexpr uint32_t kEdge = kMask + 64;               // edge class of every block (u8 [N <= 4096])
+constexpr uint32_t kBar = kEdge + 4096;
 constexpr uint32_t kSmemBytes = kBar + 256;
 
 struct Bars {
@@ -89,13 +90,11 @@ __device__ __forceinline__ uint64_t gtime() {
   return t;
 }
 
-// Bounded wait: gives up after ~2 s (nothing here legitimately waits that long), records
-// the timeout in the error word and returns false. Once any wait of the launch has run
-// out, every later wait returns at once, so a broken pipeline drains quickly instead of
-// timing out wait by wait.
-__device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint32_t* err,
-                                      bool honour_abort = true) {
-  if (tc::mbar_try_wait(bar, parity)) return true;
+// Bounded wait, slow path: polls until the phase completes or ~2 s have passed (nothing
+// here legitimately waits that long), then records the timeout in the error word and
+// returns false. Once any wait of the launch has run out, every later wait returns at
+// once, so a broken pipeline drains quickly instead of timing out wait by wait.
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, uint32_t* err, bool honour_abort) {
   const uint64_t t0 = gtime();
   while (true) {
     for (int i = 0; i < 32; ++i)
@@ -107,10 +106,11 @@ __device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint32_t* 
     }
   }
 }
-
-// Named barrier for the two softmax warps that share a TMEM lane quarter (64 threads).
-__device__ __forceinline__ void pair_sync(int quarter) {
-  asm volatile("bar.sync %0, 64;" ::"r"(quarter + 1) : "memory");
+// Fast path inline: one non-blocking test of the phase.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                         bool honour_abort = true) {
+  if (tc::mbar_test_wait(bar, parity)) return true;
+  return wait_bar_slow(bar, parity, err, honour_abort);
 }
 
 __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, int& wv) {
@@ -121,36 +121,35 @@ __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, in
   return hv * wv;
 }
 
-// One KV block of one query row half (softmax warps). Both halves of the S row from TMEM
-// (the partner's half only for the row max) -> group maxima -> alpha -> one fused loop computing
-// p448 = 2^(S c + log2 448 - m_new), the row sum and the quantised P bytes (E4M3, or E2M1
-// with an E4M3 scale per 16 keys) stored straight into the P tile -> O rescale by alpha
-// in TMEM when the max moved (after the previous P V has finished) -> P ready.
+// One KV block of one query row (softmax warps). S row from TMEM -> group maxima -> row
+// max -> alpha -> one fused loop computing p448 = 2^(S c + log2 448 - m_new), the row
+// sum and the quantised P bytes (E4M3, or E2M1 with an E4M3 scale per 16 keys) stored
+// straight into the P tile -> O rescale by alpha in TMEM when the max moved (after the
+// previous P V has landed) -> P ready.
 template <int D, int BS, bool FP8>
-__device__ __forceinline__ void softmax_block(const Geo& g, const Ws& w, Bars* bars, uint8_t* sm, uint32_t tmem,
-                                              uint32_t lane_base, float* red, int half, int quarter, int r,
-                                              int j, int bh, float sq, uint32_t gblk, int t, float& m, float& l) {
-  constexpr int HB = BS / 2, HD = D / 2, NG = HB / 16;
+__device__ __forceinline__ void softmax_block(const Ws& w, Bars* bars, uint8_t* sm, uint32_t tmem,
+                                              uint32_t lane_base, int r, float c, int ecls,
+                                              uint32_t gblk, int t, float& m, float& l) {
+  constexpr int NG = BS / 16;
   constexpr int KV4 = BS < 64 ? 64 : BS;
-  const float c = sq * w.sk[(size_t)bh * g.N + j] * g.sm_scale * kLog2e;
-  int hv, wv;
-  const bool edge = block_valid_rows(g, j, hv, wv) < BS;
   const uint32_t b = gblk & 1, pb = gblk & 1;
   wait_bar(&bars->s_full[b], (gblk >> 1) & 1, w.err);
   tc::fence_after_sync();
-  uint32_t sr[HB];
+  uint32_t sr[BS];
 #pragma unroll
-  for (int c0 = 0; c0 < HB; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColS + b * 128 + half * HB + c0, sr + c0);
+  for (int c0 = 0; c0 < BS; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColS + b * 128 + c0, sr + c0);
   tc::tmem_wait_ld();
   tc::fence_before_sync();
   tc::mbar_arrive(&bars->s_free[b]);
   float* s = reinterpret_cast<float*>(sr);
-  if (edge) {
+  if (ecls != 0) {                                        // padded slots of an edge block
+    const uint32_t* mw = reinterpret_cast<const uint32_t*>(sm + kMask) + ecls * 4;
 #pragma unroll
-    for (int k = 0; k < HB; ++k) {
-      const int kk = half * HB + k;
-      const int ky = kk / g.pw, kx = kk - ky * g.pw;
-      if (!(ky < hv && kx < wv)) s[k] = -INFINITY;
+    for (int q = 0; q < BS / 32; ++q) {
+      const uint32_t bits = mw[q];
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (!((bits >> e) & 1u)) s[32 * q + e] = -INFINITY;
     }
   }
   // group maxima of the raw dot products (c > 0, so they order like S)
@@ -164,10 +163,7 @@ __device__ __forceinline__ void softmax_block(const Geo& g, const Ws& w, Bars* b
   float mh = gm[0];
 #pragma unroll
   for (int q = 1; q < NG; ++q) mh = fmaxf(mh, gm[q]);
-  float* rp = red + (gblk & 1) * 256;
-  rp[half * 128 + r] = mh * c;
-  pair_sync(quarter);
-  const float m_new = fmaxf(m, fmaxf(rp[r], rp[128 + r]));
+  const float m_new = fmaxf(m, mh * c);
   const float alpha = ex2(m - m_new);
   const float bias = kLog2_448 - m_new;
   // the P buffer is free once the P V two blocks back has completed
@@ -188,13 +184,14 @@ __device__ __forceinline__ void softmax_block(const Geo& g, const Ws& w, Bars* b
         }
         wd[e / 4] = (uint32_t)f32x2_to_e4m3x2(p[0], p[1]) | ((uint32_t)f32x2_to_e4m3x2(p[2], p[3]) << 16);
       }
-      *reinterpret_cast<uint4*>(pbuf + kPData + kmajor_off(r, half * HB + 16 * q, BS)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      *reinterpret_cast<uint4*>(pbuf + kPData + kmajor_off(r, 16 * q, BS)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
     }
   } else {
-    uint8_t* sfrow = pbuf + kPSF + (r & 31) * 16 + (r >> 5) * 4;
+    uint32_t sfw[KV4 / 64];
+#pragma unroll
+    for (int q = 0; q < KV4 / 64; ++q) sfw[q] = 0u;
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
-      const int gk = half * HB + 16 * q;                 // first key of the group
       // group scale from the group max: sigma = E4M3(448 p_max / 6)
       uint32_t sc = f32_to_e4m3(ex2(fmaf(gm[q], c, bias)) * (1.0f / 6.0f));
       const float sg = e4m3_to_f32((uint8_t)sc);
@@ -206,34 +203,33 @@ __device__ __forceinline__ void softmax_block(const Geo& g, const Ws& w, Bars* b
         sum4[e & 3] += p;
         y[e] = p * rs;
       }
-      const uint2 pk = make_uint2(f32x8_to_e2m1x8(y), f32x8_to_e2m1x8(y + 8));
-      *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, gk / 2, KV4 / 2)) = pk;
-      sfrow[(gk >> 6) * 512 + ((gk >> 4) & 3)] = (uint8_t)sc;
+      *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, 8 * q, KV4 / 2)) =
+          make_uint2(f32x8_to_e2m1x8(y), f32x8_to_e2m1x8(y + 8));
+      sfw[q >> 2] |= sc << (8 * (q & 3));
     }
-    if (KV4 > BS && half == 1) {                           // zero keys past the block (32-token blocks)
 #pragma unroll
-      for (int gk = BS; gk < KV4; gk += 16) {
-        *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, gk / 2, KV4 / 2)) = make_uint2(0u, 0u);
-        sfrow[(gk >> 6) * 512 + ((gk >> 4) & 3)] = 0;
-      }
-    }
+    for (int gk = BS; gk < KV4; gk += 16)                  // zero keys past the block (32-token blocks)
+      *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, gk / 2, KV4 / 2)) = make_uint2(0u, 0u);
+#pragma unroll
+    for (int q = 0; q < KV4 / 64; ++q)
+      *reinterpret_cast<uint32_t*>(pbuf + kPSF + q * 512 + (r & 31) * 16 + (r >> 5) * 4) = sfw[q];
   }
   l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
-  // O rows of this warp's half *= alpha, once the previous P V has landed
+  // O row *= alpha, once the previous P V has landed
   if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
     const uint32_t gp = gblk - 1;
     wait_bar(&bars->p_free[gp & 1], (gp >> 1) & 1, w.err);
     tc::fence_after_sync();
 #pragma unroll
-    for (int h0 = 0; h0 < HD; h0 += 32) {
+    for (int h0 = 0; h0 < D; h0 += 32) {
       uint32_t orr[32];
-      tc::tmem_ld16(tmem + lane_base + kColO + half * HD + h0, orr);
-      tc::tmem_ld16(tmem + lane_base + kColO + half * HD + h0 + 16, orr + 16);
+      tc::tmem_ld16(tmem + lane_base + kColO + h0, orr);
+      tc::tmem_ld16(tmem + lane_base + kColO + h0 + 16, orr + 16);
       tc::tmem_wait_ld();
 #pragma unroll
       for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-      tc::tmem_st16(tmem + lane_base + kColO + half * HD + h0, orr);
-      tc::tmem_st16(tmem + lane_base + kColO + half * HD + h0 + 16, orr + 16);
+      tc::tmem_st16(tmem + lane_base + kColO + h0, orr);
+      tc::tmem_st16(tmem + lane_base + kColO + h0 + 16, orr + 16);
     }
     tc::tmem_wait_st();
   }
@@ -274,6 +270,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
   }
   for (uint32_t o = tid * 16; o < kStage0; o += kThreads * 16)
     *reinterpret_cast<uint4*>(sm + o) = make_uint4(0u, 0u, 0u, 0u);
+  // Edge tables: class of each block (bit 1: last window row is short, bit 0: last window
+  // column is short) and, per class, which of the BS slots hold real tokens.
+  {
+    const int hl = g.Hf - (g.ny - 1) * g.ph, wl = g.Wf - (g.nx - 1) * g.pw;
+    uint8_t* ecl = sm + kEdge;
+    for (int n = tid; n < N; n += kThreads) {
+      const int rem = n % (g.ny * g.nx), by = rem / g.nx, bx = rem - by * g.nx;
+      ecl[n] = (uint8_t)(((by == g.ny - 1 && hl < g.ph) ? 2 : 0) | ((bx == g.nx - 1 && wl < g.pw) ? 1 : 0));
+    }
+    if (tid < 16) {
+      const int cls = tid >> 2, q = tid & 3;
+      const int hv = (cls & 2) ? hl : g.ph, wv = (cls & 1) ? wl : g.pw;
+      uint32_t bits = 0u;
+      for (int e = 0; e < 32; ++e) {
+        const int k = 32 * q + e, ky = k / g.pw, kx = k - ky * g.pw;
+        if (k < BS && ky < hv && kx < wv) bits |= 1u << e;
+      }
+      reinterpret_cast<uint32_t*>(sm + kMask)[tid] = bits;
+    }
+  }
   if (warp == kMmaWarp) {
     tc::tmem_alloc(&bars->tmem, 512);
     tc::tmem_relinquish();
@@ -424,17 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       wait_bar(&bars->done, 0, w.err, false);   // all MMAs retired before TMEM is freed
     }
   } else {
-    // ===================== softmax + epilogue (warps 0-7) =====================
-    // Warps w and w+4 share TMEM lane quarter w%4 (query rows 32(w%4) .. +31); warp
-    // w/4 = h takes key columns [h BS/2, (h+1) BS/2) of S and P and output columns
-    // [h D/2, (h+1) D/2) of O. The row max of each block and the final row sum are
-    // exchanged through shared memory under a named barrier of the pair.
-    constexpr int HB = BS / 2, HD = D / 2;
-    const int quarter = warp & 3, half = warp >> 2;
-    const int r = quarter * 32 + lane;                   // query row = TMEM lane
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    float* red = reinterpret_cast<float*>(sm + kRed);
-    float* lx = reinterpret_cast<float*>(sm + kLx);
+    // ===================== softmax + epilogue (warps 0-3) =====================
+    const int r = tid;                                   // query row = TMEM lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const int fpf = g.ny * g.nx;
     uint32_t gblk = 0, wi = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x, ++wi) {
@@ -447,56 +455,71 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       __nv_bfloat16* orow = nullptr;
       if (row_ok) {
         const int f = i / fpf, rem = i - f * fpf, by = rem / g.nx, bx = rem - by * g.nx;
-        const size_t t = (size_t)f * g.Hf * g.Wf + (size_t)(by * g.ph + wy) * g.Wf + bx * g.pw + wx;
-        orow = out + ((size_t)bh * g.T + t) * D + half * HD;
+        const size_t tk = (size_t)f * g.Hf * g.Wf + (size_t)(by * g.ph + wy) * g.Wf + bx * g.pw + wx;
+        orow = out + ((size_t)bh * g.T + tk) * D;
       }
       if (nb == 0) {
         if (row_ok)
-          for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0u, 0u, 0u, 0u);
+          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0u, 0u, 0u, 0u);
         continue;
       }
       const float sq = w.sq[qi];
       const int16_t* l8 = w.list8 + qi * w.n8s;
       const int16_t* l4 = w.list4 + qi * w.n4s;
       float m = -INFINITY, l = 0.0f;
+      // block index j, logit scale c and edge geometry of each visited block, fetched two
+      // (list entry) and one (scale) blocks ahead; raw list entries are clamped only
+      // where they are used, so that the loads stay in flight across the block
+      const float cq = sq * g.sm_scale * kLog2e;
+      const float* skh = w.sk + (size_t)bh * N;
+      auto list_raw = [&](int t) -> int { return t < n8 ? l8[t] : l4[t - n8]; };
+      auto clampj = [&](int j) -> int { return (j < 0 || j >= N) ? 0 : j; };
+      int j_next = nb > 1 ? list_raw(1) : 0;
+      int j_cur = clampj(list_raw(0));
+      float sk_cur = skh[j_cur];
       for (int t = 0; t < nb; ++t, ++gblk) {
-        int j = t < n8 ? l8[t] : l4[t - n8];
-        if (j < 0 || j >= N) j = 0;
+        const int j_after = t + 2 < nb ? list_raw(t + 2) : 0;
+        const int jn = clampj(j_next);
+        const float sk_next = skh[jn];
+        const int ecls = sm[kEdge + j_cur];
+        const float c = cq * sk_cur;
         if (t < n8)
-          softmax_block<D, BS, true>(g, w, bars, sm, tmem, lane_base, red, half, quarter, r, j, bh, sq, gblk, t, m, l);
+          softmax_block<D, BS, true>(w, bars, sm, tmem, lane_base, r, c, ecls, gblk, t, m, l);
         else
-          softmax_block<D, BS, false>(g, w, bars, sm, tmem, lane_base, red, half, quarter, r, j, bh, sq, gblk, t, m, l);
+          softmax_block<D, BS, false>(w, bars, sm, tmem, lane_base, r, c, ecls, gblk, t, m, l);
+        j_cur = jn;
+        sk_cur = sk_next;
+        j_next = j_after;
       }
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
-      lx[half * 128 + r] = l;
-      pair_sync(quarter);
-      const float lt = lx[r] + lx[128 + r];          // 448 * row sum
       wait_bar(&bars->o_full, wi & 1, w.err);
       tc::fence_after_sync();
-      const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-      const float* sv = w.sv + (size_t)bh * D + half * HD;
-      uint32_t rr[HD];
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;     // l holds 448 * row sum
+      const float* sv = w.sv + (size_t)bh * D;
 #pragma unroll
-      for (int c0 = 0; c0 < HD; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColO + half * HD + c0, rr + c0);
-      tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      tc::mbar_arrive(&bars->o_free);
-      if (row_ok) {
+      for (int h0 = 0; h0 < D; h0 += 64) {
+        uint32_t rr[64];
 #pragma unroll
-        for (int c0 = 0; c0 < HD; c0 += 8) {
-          uint32_t pk[4];
+        for (int c0 = 0; c0 < 64; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColO + h0 + c0, rr + c0);
+        tc::tmem_wait_ld();
+        if (row_ok) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int cc = c0 + 2 * e;
-            const float a = __uint_as_float(rr[cc]) * __ldg(sv + cc) * inv;
-            const float bq = __uint_as_float(rr[cc + 1]) * __ldg(sv + cc + 1) * inv;
-            const __nv_bfloat162 hh = __floats2bfloat162_rn(a, bq);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&hh);
+          for (int c0 = 0; c0 < 64; c0 += 8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int cc = h0 + c0 + 2 * e;
+              const float a = __uint_as_float(rr[c0 + 2 * e]) * __ldg(sv + cc) * inv;
+              const float bq = __uint_as_float(rr[c0 + 2 * e + 1]) * __ldg(sv + cc + 1) * inv;
+              const __nv_bfloat162 hh = __floats2bfloat162_rn(a, bq);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
+            *reinterpret_cast<uint4*>(orow + h0 + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-          *reinterpret_cast<uint4*>(orow + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
-      pair_sync(quarter);                            // lx is reused by the next work item
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars->o_free);
     }
   }
   tc::fence_before_sync();
