@@ -138,7 +138,8 @@ __device__ __forceinline__ void softmax_block(const Ws& w, Bars* bars, uint8_t* 
   uint32_t sr[BS];
 #pragma unroll
   for (int c0 = 0; c0 < BS; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColS + b * 128 + c0, sr + c0);
-  tc::tmem_wait_ld();
+#pragma unroll
+  for (int c0 = 0; c0 < BS; c0 += 16) tc::tmem_wait_ld16(sr + c0);
   tc::fence_before_sync();
   tc::mbar_arrive(&bars->s_free[b]);
   float* s = reinterpret_cast<float*>(sr);
@@ -225,7 +226,8 @@ __device__ __forceinline__ void softmax_block(const Ws& w, Bars* bars, uint8_t* 
       uint32_t orr[32];
       tc::tmem_ld16(tmem + lane_base + kColO + h0, orr);
       tc::tmem_ld16(tmem + lane_base + kColO + h0 + 16, orr + 16);
-      tc::tmem_wait_ld();
+      tc::tmem_wait_ld16(orr);
+      tc::tmem_wait_ld16(orr + 16);
 #pragma unroll
       for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
       tc::tmem_st16(tmem + lane_base + kColO + h0, orr);
@@ -501,7 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         uint32_t rr[64];
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColO + h0 + c0, rr + c0);
-        tc::tmem_wait_ld();
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) tc::tmem_wait_ld16(rr + c0);
         if (row_ok) {
 #pragma unroll
           for (int c0 = 0; c0 < 64; c0 += 8) {
