@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
   __nv_bfloat16* X = reinterpret_cast<__nv_bfloat16*>(smem);
   const int bs = g.bs;
   uint8_t* sfbuf = smem + (size_t)bs * RS * 2;             // up to 1 KB of group scales
-  float* red = reinterpret_cast<float*>(sfbuf + 1024);      // 8 floats of reduction scratch
+  float* red = reinterpret_cast<float*>(sfbuf + 1024);      // reduction scratch / V scales
 
   const int n = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int tid = threadIdx.x;
@@ -85,15 +85,25 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
 
   // stage the window (padded slots zero)
   const __nv_bfloat16* sbase = src + (size_t)bh * g.T * D;
-  for (int u = tid; u < bs * VPR; u += 256) {
-    const int s = u / VPR, cv = u - s * VPR;
-    const int wy = s / g.pw, wx = s - wy * g.pw;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (wy < hv && wx < wv) {
-      const size_t t = (size_t)f * g.Hf * g.Wf + (size_t)(y0 + wy) * g.Wf + (x0 + wx);
-      val = ld_stream_u4(sbase + t * D + cv * 8);
+  {
+    // slot s = wy*pw + wx advances by a fixed step per iteration: step the window
+    // coordinates instead of dividing every time
+    constexpr int DS = 256 / VPR;
+    const int cv = tid % VPR;
+    int s0 = tid / VPR;
+    int wy = s0 / g.pw, wx = s0 - wy * g.pw;
+    const int dy = DS / g.pw, dx = DS - dy * g.pw;
+    for (int sl = s0; sl < bs; sl += DS) {
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (wy < hv && wx < wv) {
+        const size_t t = (size_t)f * g.Hf * g.Wf + (size_t)(y0 + wy) * g.Wf + (x0 + wx);
+        val = ld_stream_u4(sbase + t * D + cv * 8);
+      }
+      *reinterpret_cast<uint4*>(X + sl * RS + cv * 8) = val;
+      wx += dx;
+      wy += dy;
+      if (wx >= g.pw) { wx -= g.pw; ++wy; }
     }
-    *reinterpret_cast<uint4*>(X + s * RS + cv * 8) = val;
   }
   const int sfbytes = which < 2 ? (int)w.sf_qk : (int)w.sf_v;
   for (int i = tid; i < sfbytes / 4; i += 256) reinterpret_cast<uint32_t*>(sfbuf)[i] = 0u;
@@ -101,21 +111,37 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
 
   if (which < 2) {
     // ---- draft pooling: fp32 running sum in slot order, then IEEE divide; exact max ----
+    // threads [0, D/2): sums of channel pairs; [D/2, D): maxima of channel pairs
     float* avg_out = (which == 0 ? w.qavg : w.kavg) + ((size_t)bh * g.N + n) * D;
     float* max_out = (which == 0 ? w.qmax : w.kmax) + ((size_t)bh * g.N + n) * D;
-    if (tid < 2 * D) {
-      const int c = tid % D;
-      const bool do_sum = tid < D;
-      float acc = do_sum ? 0.0f : -INFINITY;
-      for (int s = 0; s < bs; ++s) {
-        const int wy = s / g.pw, wx = s - wy * g.pw;
-        if (wy < hv && wx < wv) {
-          const float x = __bfloat162float(X[s * RS + c]);
-          acc = do_sum ? __fadd_rn(acc, x) : fmaxf(acc, x);
+    if (tid < D) {
+      const bool do_sum = tid < D / 2;
+      const int c2 = 2 * (tid % (D / 2));
+      float a0 = do_sum ? 0.0f : -INFINITY, a1 = a0;
+      for (int wy = 0; wy < hv; ++wy) {
+        const __nv_bfloat16* row = X + wy * g.pw * RS + c2;
+        if (do_sum) {
+#pragma unroll 4
+          for (int wx = 0; wx < wv; ++wx) {
+            const uint32_t u = *reinterpret_cast<const uint32_t*>(row + wx * RS);
+            a0 = __fadd_rn(a0, __uint_as_float(u << 16));
+            a1 = __fadd_rn(a1, __uint_as_float(u & 0xFFFF0000u));
+          }
+        } else {
+#pragma unroll 4
+          for (int wx = 0; wx < wv; ++wx) {
+            const uint32_t u = *reinterpret_cast<const uint32_t*>(row + wx * RS);
+            a0 = fmaxf(a0, __uint_as_float(u << 16));
+            a1 = fmaxf(a1, __uint_as_float(u & 0xFFFF0000u));
+          }
         }
       }
-      if (do_sum) avg_out[c] = __fdiv_rn(acc, (float)(hv * wv));
-      else max_out[c] = acc;
+      if (do_sum) {
+        const float cnt = (float)(hv * wv);
+        *reinterpret_cast<float2*>(avg_out + c2) = make_float2(__fdiv_rn(a0, cnt), __fdiv_rn(a1, cnt));
+      } else {
+        *reinterpret_cast<float2*>(max_out + c2) = make_float2(a0, a1);
+      }
     }
     // ---- block amax -> outer scale ----
     float am = 0.0f;
@@ -168,9 +194,13 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
   } else {
     // ---- V: per-channel outer scale from the amax pre-pass; tiles are channel-major ----
     const float* am = w.vamax + (size_t)bh * D;
-    if (n == 0)
-      for (int c = tid; c < D; c += 256)
-        w.sv[(size_t)bh * D + c] = am[c] > 0.0f ? __fdiv_rn(am[c], kE4M3Max) : 1.0f;
+    float* vinv = red;                                      // D inverse channel scales
+    for (int c = tid; c < D; c += 256) {
+      const float a = am[c];
+      vinv[c] = a > 0.0f ? __fdiv_rn(kE4M3Max, a) : 1.0f;
+      if (n == 0) w.sv[(size_t)bh * D + c] = a > 0.0f ? __fdiv_rn(a, kE4M3Max) : 1.0f;
+    }
+    __syncthreads();
     uint8_t* t8 = w.v8 + ((size_t)bh * g.N + n) * w.tile8_v;
     uint8_t* t4 = w.v4 + ((size_t)bh * g.N + n) * w.tile4_v;
     const int SC = bs / 16, SC4 = g.kv4 / 16;
@@ -178,8 +208,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
       const int cg = u / (8 * SC4), within = u - cg * 8 * SC4;
       const int sc = within >> 3, cc = within & 7;
       const int c = cg * 8 + cc;
-      const float a = am[c];
-      const float inv = a > 0.0f ? __fdiv_rn(kE4M3Max, a) : 1.0f;
+      const float inv = vinv[c];
       float y[16];
       if (sc < SC) {
 #pragma unroll
@@ -207,7 +236,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
 }
 
 size_t prepare_smem_bytes(const Geo& g) {
-  return (size_t)g.bs * (g.d + 8) * 2 + 1024 + 64;
+  return (size_t)g.bs * (g.d + 8) * 2 + 1024 + 4 * 128;
 }
 
 cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
