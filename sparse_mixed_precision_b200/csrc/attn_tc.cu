@@ -18,14 +18,19 @@
 //   O += P~ V_j'             same MMA kind as the block, accumulating into the one O.
 // Epilogue: out = O s_v / (448 l) in bf16, written to the tokens' original positions.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work items in head-major
-// order so that one head's K/V stay in L2):
-//   warps 0-3  softmax + epilogue: thread r owns query row r (TMEM lane r), all key
-//              columns of S / P and all output columns of O; one softmax warp per SM
-//              sub-partition, so its short per-block bookkeeping never competes for
-//              issue slots with another warp's exponential loop
-//   warp 4     MMA issue (one thread) and TMEM allocation
-//   warp 5     producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
+// Two query tiles (work items) per CTA, processed as a ping-pong: while one tile's
+// softmax warpgroup runs its exponential loop, the other's does its per-block
+// bookkeeping, so the SM's special-function units and issue slots stay busy. 384 threads,
+// one CTA per SM, persistent over work items in head-major order (one head's K/V stay in
+// L2); round k of a CTA takes its work items 2k (tile A) and 2k+1 (tile B):
+//   warps 0-3   softmax + epilogue of tile A: thread r owns query row r (TMEM lane r)
+//   warps 4-7   softmax + epilogue of tile B
+//   warp 8      MMA issue (one thread) and TMEM allocation
+//   warp 9      producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
+//   warps 10-11 idle
+// Tensor memory: O of each tile, ONE S region the two tiles take in turns, and scale
+// factors. MMA order: S_A(0), S_B(0), then per block t: PV_A(t), S_A(t+1), PV_B(t),
+// S_B(t+1); K/V stages are filled and released in that order.
 // Every mbarrier wait is bounded; a wait that runs out sets the workspace error word and
 // the kernel carries on to a clean exit.
 #include "common.cuh"
@@ -34,10 +39,9 @@
 namespace da2 {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;   // warps 0-3
-constexpr int kMmaWarp = 4;
-constexpr int kLoadWarp = 5;
+constexpr int kThreads = 384;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
 constexpr int kStages = 4;
 constexpr int kPrefetch = 8;   // KV blocks the producer warms in L2 ahead of its copies
 constexpr float kLog2e = 1.4426950408889634f;
@@ -59,27 +63,29 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-// TMEM columns (512 allocated)
-constexpr uint32_t kColO = 0, kColS = 128, kColSFQ = 384, kColSFK = 392, kColSFP = 408,
-                   kColSFV = 424;
+// TMEM columns (512 allocated): O of tile A and B, the shared S region, scale factors.
+constexpr uint32_t kColO0 = 0, kColO1 = 128, kColS = 256;
+constexpr uint32_t kColSFQ = 384, kColSFK = 400, kColSFP = 416, kColSFV = 432;   // + 8 * tile
 
 // shared memory carve-up (bytes)
-constexpr uint32_t kQ8 = 0;                       // 128 x 128 E4M3
-constexpr uint32_t kQ4 = kQ8 + 16384;             // 128 x 64 bytes E2M1
-constexpr uint32_t kSFQ = kQ4 + 8192;             // 2 scale atoms
-constexpr uint32_t kStage0 = kSFQ + 1024;
+constexpr uint32_t kQ8 = 0, kQ4 = 16384, kSFQ = 24576, kQBytes = 25600;   // per tile
+constexpr uint32_t kStage0 = 2 * kQBytes;
 constexpr uint32_t kStK = 0, kStV = 16384, kStSFK = 32768, kStSFV = 33792, kStageBytes = 34816;
 constexpr uint32_t kP0 = kStage0 + kStages * kStageBytes;
-constexpr uint32_t kPData = 0, kPSF = 16384, kPBytes = 17408;
+constexpr uint32_t kPData = 0, kPSF = 16384, kPBytes = 17408;                 // per tile
 constexpr uint32_t kMask = kP0 + 2 * kPBytes;      // 4 slot-validity masks x 4 words
-constexpr uint32_t kEdge = kMask + 64;               // edge class of every block (u8 [N <= 4096])
+constexpr uint32_t kEdge = kMask + 64;             // edge class of every block (u8 [N <= 4096])
 constexpr uint32_t kBar = kEdge + 4096;
 constexpr uint32_t kSmemBytes = kBar + 256;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
+struct TileBars {
+  uint64_t s_full, s_free, p_full, p_free, q_full, q_empty, o_full, o_free;
+};
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full[2], p_free[2];
-  uint64_t q_full, q_empty, o_full, o_free, done;
+  TileBars tb[2];
+  uint64_t done;
   uint32_t tmem;
 };
 static_assert(sizeof(Bars) <= 256, "barrier area");
@@ -121,27 +127,28 @@ __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, in
   return hv * wv;
 }
 
-// One KV block of one query row (softmax warps). S row from TMEM -> group maxima -> row
-// max -> alpha -> one fused loop computing p448 = 2^(S c + log2 448 - m_new), the row
-// sum and the quantised P bytes (E4M3, or E2M1 with an E4M3 scale per 16 keys) stored
-// straight into the P tile -> O rescale by alpha in TMEM when the max moved (after the
+// One KV block of one query row of a tile (softmax warps). The S row is read once from
+// the shared S region (which is released at once) -> group maxima -> row max -> alpha ->
+// one fused loop computing p448 = 2^(S c + log2 448 - m_new), the row sum and the
+// quantised P bytes (E4M3, or E2M1 with an E4M3 scale per 16 keys) stored straight into
+// the tile's P buffer -> O rescale by alpha in TMEM when the max moved (after the tile's
 // previous P V has landed) -> P ready.
+// gx counts this tile's blocks over the whole launch.
 template <int D, int BS, bool FP8>
-__device__ __forceinline__ void softmax_block(const Ws& w, Bars* bars, uint8_t* sm, uint32_t tmem,
-                                              uint32_t lane_base, int r, float c, int ecls,
-                                              uint32_t gblk, int t, float& m, float& l) {
+__device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t* sm, uint8_t* pbuf,
+                                              uint32_t tmem, uint32_t lane_base, uint32_t colO, int r,
+                                              float c, int ecls, uint32_t gx, int t, float& m, float& l) {
   constexpr int NG = BS / 16;
   constexpr int KV4 = BS < 64 ? 64 : BS;
-  const uint32_t b = gblk & 1, pb = gblk & 1;
-  wait_bar(&bars->s_full[b], (gblk >> 1) & 1, w.err);
+  wait_bar(&tb->s_full, gx & 1, w.err);
   tc::fence_after_sync();
   uint32_t sr[BS];
 #pragma unroll
-  for (int c0 = 0; c0 < BS; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColS + b * 128 + c0, sr + c0);
+  for (int c0 = 0; c0 < BS; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColS + c0, sr + c0);
 #pragma unroll
   for (int c0 = 0; c0 < BS; c0 += 16) tc::tmem_wait_ld16(sr + c0);
   tc::fence_before_sync();
-  tc::mbar_arrive(&bars->s_free[b]);
+  tc::mbar_arrive(&tb->s_free);                          // the S region may be reused
   float* s = reinterpret_cast<float*>(sr);
   if (ecls != 0) {                                        // padded slots of an edge block
     const uint32_t* mw = reinterpret_cast<const uint32_t*>(sm + kMask) + ecls * 4;
@@ -167,9 +174,11 @@ __device__ __forceinline__ void softmax_block(const Ws& w, Bars* bars, uint8_t* 
   const float m_new = fmaxf(m, mh * c);
   const float alpha = ex2(m - m_new);
   const float bias = kLog2_448 - m_new;
-  // the P buffer is free once the P V two blocks back has completed
-  if (gblk >= 2) wait_bar(&bars->p_free[pb], ((gblk >> 1) & 1) ^ 1, w.err);
-  uint8_t* pbuf = sm + kP0 + pb * kPBytes;
+  // the P buffer (and O) are free once this tile's previous P V has completed
+  if (t > 0) {
+    wait_bar(&tb->p_free, (gx - 1) & 1, w.err);
+    tc::fence_after_sync();
+  }
   float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (FP8) {
 #pragma unroll
@@ -216,29 +225,26 @@ __device__ __forceinline__ void softmax_block(const Ws& w, Bars* bars, uint8_t* 
       *reinterpret_cast<uint32_t*>(pbuf + kPSF + q * 512 + (r & 31) * 16 + (r >> 5) * 4) = sfw[q];
   }
   l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
-  // O row *= alpha, once the previous P V has landed
+  // O row *= alpha (the previous P V of this tile has landed: waited above)
   if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-    const uint32_t gp = gblk - 1;
-    wait_bar(&bars->p_free[gp & 1], (gp >> 1) & 1, w.err);
-    tc::fence_after_sync();
 #pragma unroll
     for (int h0 = 0; h0 < D; h0 += 32) {
       uint32_t orr[32];
-      tc::tmem_ld16(tmem + lane_base + kColO + h0, orr);
-      tc::tmem_ld16(tmem + lane_base + kColO + h0 + 16, orr + 16);
+      tc::tmem_ld16(tmem + lane_base + colO + h0, orr);
+      tc::tmem_ld16(tmem + lane_base + colO + h0 + 16, orr + 16);
       tc::tmem_wait_ld16(orr);
       tc::tmem_wait_ld16(orr + 16);
 #pragma unroll
       for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-      tc::tmem_st16(tmem + lane_base + kColO + h0, orr);
-      tc::tmem_st16(tmem + lane_base + kColO + h0 + 16, orr + 16);
+      tc::tmem_st16(tmem + lane_base + colO + h0, orr);
+      tc::tmem_st16(tmem + lane_base + colO + h0 + 16, orr + 16);
     }
     tc::tmem_wait_st();
   }
   m = m_new;
   tc::fence_proxy_async_smem();
   tc::fence_before_sync();
-  tc::mbar_arrive(&bars->p_full[pb]);
+  tc::mbar_arrive(&tb->p_full);
 }
 
 template <int D, int BS>
@@ -250,23 +256,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
   const int n8 = g.n8, nb = g.n8 + g.n4;
   const int total = BH * N;
   constexpr int KV4 = BS < 64 ? 64 : BS;
+  // work items of this CTA: blockIdx.x + m gridDim.x; round k takes m = 2k (A), 2k+1 (B)
+  const int my_items = (int)blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int rounds = (my_items + 1) / 2;
+  auto item_of = [&](int k, int x) { return (int)blockIdx.x + (2 * k + x) * (int)gridDim.x; };
+  auto has_tile = [&](int k, int x) { return 2 * k + x < my_items; };
 
-  // ---- set-up: barriers, zeroed Q tiles (rows >= bs stay zero), TMEM ----
+  // ---- set-up: barriers, zeroed Q tiles (rows >= bs stay zero), edge tables, TMEM ----
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&bars->kv_full[s], 1);
       tc::mbar_init(&bars->kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(&bars->s_full[b], 1);
-      tc::mbar_init(&bars->s_free[b], kSoftmaxThreads);
-      tc::mbar_init(&bars->p_full[b], kSoftmaxThreads);
-      tc::mbar_init(&bars->p_free[b], 1);
+    for (int x = 0; x < 2; ++x) {
+      TileBars* tb = &bars->tb[x];
+      tc::mbar_init(&tb->s_full, 1);
+      tc::mbar_init(&tb->s_free, 128);
+      tc::mbar_init(&tb->p_full, 128);
+      tc::mbar_init(&tb->p_free, 1);
+      tc::mbar_init(&tb->q_full, 1);
+      tc::mbar_init(&tb->q_empty, 1);
+      tc::mbar_init(&tb->o_full, 1);
+      tc::mbar_init(&tb->o_free, 128);
     }
-    tc::mbar_init(&bars->q_full, 1);
-    tc::mbar_init(&bars->q_empty, 1);
-    tc::mbar_init(&bars->o_full, 1);
-    tc::mbar_init(&bars->o_free, kSoftmaxThreads);
     tc::mbar_init(&bars->done, 1);
     tc::fence_mbar_init();
   }
@@ -302,14 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem;
 
+  if (warp >= 8) {
   if (warp == kLoadWarp) {
     // ===================== producer =====================
-    if (lane == 0) {
-      uint32_t gblk = 0, wi = 0;
-      auto kv_prefetch = [&](int bh, const int16_t* l8, const int16_t* l4, int t) {
-        const bool fp8 = t < n8;
-        int j = fp8 ? l8[t] : l4[t - n8];
-        if (j < 0 || j >= N) j = 0;
+    if (lane == 0 && nb > 0) {
+      uint32_t gkv = 0;
+      auto list_j = [&](const int16_t* l8, const int16_t* l4, int t) {
+        const int j = t < n8 ? l8[t] : l4[t - n8];
+        return (j < 0 || j >= N) ? 0 : j;
+      };
+      auto kv_prefetch = [&](int bh, int j, bool fp8) {
         const size_t kj = (size_t)bh * N + j;
         if (fp8) {
           tc::prefetch_l2(w.k8 + kj * w.tile8_qk, BS * D);
@@ -319,135 +333,165 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           tc::prefetch_l2(w.v4 + kj * w.tile4_v, D * KV4 / 2);
         }
       };
-      for (int item = blockIdx.x; item < total; item += gridDim.x, ++wi) {
-        if (nb == 0) continue;
-        const int bh = item / N, i = item - bh * N;
-        const size_t qi = (size_t)bh * N + i;
-        const int16_t* l8 = w.list8 + qi * w.n8s;
-        const int16_t* l4 = w.list4 + qi * w.n4s;
-        for (int t = 0; t < kPrefetch && t < nb; ++t) kv_prefetch(bh, l8, l4, t);
-        wait_bar(&bars->q_empty, (wi & 1) ^ 1, w.err);
-        const uint32_t qbytes = BS * D + BS * D / 2 + (uint32_t)w.sf_qk;
-        tc::mbar_arrive_expect_tx(&bars->q_full, qbytes);
-        tc::bulk_g2s(sm + kQ8, w.q8 + qi * w.tile8_qk, BS * D, &bars->q_full);
-        tc::bulk_g2s(sm + kQ4, w.q4 + qi * w.tile4_qk, BS * D / 2, &bars->q_full);
-        tc::bulk_g2s(sm + kSFQ, w.sfq4 + qi * w.sf_qk, (uint32_t)w.sf_qk, &bars->q_full);
-        const int nxt = item + gridDim.x;             // warm L2 with the next work item's Q
-        if (nxt < total) {
-          const size_t qn = (size_t)(nxt / N) * N + (nxt % N);
-          tc::prefetch_l2(w.q8 + qn * w.tile8_qk, BS * D);
-          tc::prefetch_l2(w.q4 + qn * w.tile4_qk, BS * D / 2);
+      for (int k = 0; k < rounds; ++k) {
+        const int nx = has_tile(k, 1) ? 2 : 1;
+        int bhx[2], ix[2];
+        const int16_t* l8x[2];
+        const int16_t* l4x[2];
+        for (int x = 0; x < nx; ++x) {
+          const int item = item_of(k, x);
+          bhx[x] = item / N;
+          ix[x] = item - bhx[x] * N;
+          const size_t qi = (size_t)bhx[x] * N + ix[x];
+          l8x[x] = w.list8 + qi * w.n8s;
+          l4x[x] = w.list4 + qi * w.n4s;
+          TileBars* tb = &bars->tb[x];
+          wait_bar(&tb->q_empty, (k & 1) ^ 1, w.err);
+          const uint32_t qbytes = BS * D + BS * D / 2 + (uint32_t)w.sf_qk;
+          uint8_t* qs = sm + x * kQBytes;
+          tc::mbar_arrive_expect_tx(&tb->q_full, qbytes);
+          tc::bulk_g2s(qs + kQ8, w.q8 + qi * w.tile8_qk, BS * D, &tb->q_full);
+          tc::bulk_g2s(qs + kQ4, w.q4 + qi * w.tile4_qk, BS * D / 2, &tb->q_full);
+          tc::bulk_g2s(qs + kSFQ, w.sfq4 + qi * w.sf_qk, (uint32_t)w.sf_qk, &tb->q_full);
         }
-        for (int t = 0; t < nb; ++t, ++gblk) {
-          if (t + kPrefetch < nb) kv_prefetch(bh, l8, l4, t + kPrefetch);
+        for (int t = 0; t < kPrefetch / 2 && t < nb; ++t)
+          for (int x = 0; x < nx; ++x) kv_prefetch(bhx[x], list_j(l8x[x], l4x[x], t), t < n8);
+        for (int t = 0; t < nb; ++t) {
           const bool fp8 = t < n8;
-          int j = fp8 ? l8[t] : l4[t - n8];
-          if (j < 0 || j >= N) { set_error(w.err, kErrBadIndex); j = 0; }
-          const size_t kj = (size_t)bh * N + j;
-          const uint32_t s = gblk % kStages, k = gblk / kStages;
-          wait_bar(&bars->kv_empty[s], (k & 1) ^ 1, w.err);
-          uint8_t* st = sm + kStage0 + s * kStageBytes;
-          if (fp8) {
-            tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * BS * D);
-            tc::bulk_g2s(st + kStK, w.k8 + kj * w.tile8_qk, BS * D, &bars->kv_full[s]);
-            tc::bulk_g2s(st + kStV, w.v8 + kj * w.tile8_v, BS * D, &bars->kv_full[s]);
-          } else {
-            const uint32_t bytes = BS * D / 2 + D * KV4 / 2 + (uint32_t)w.sf_qk + (uint32_t)w.sf_v;
-            tc::mbar_arrive_expect_tx(&bars->kv_full[s], bytes);
-            tc::bulk_g2s(st + kStK, w.k4 + kj * w.tile4_qk, BS * D / 2, &bars->kv_full[s]);
-            tc::bulk_g2s(st + kStV, w.v4 + kj * w.tile4_v, D * KV4 / 2, &bars->kv_full[s]);
-            tc::bulk_g2s(st + kStSFK, w.sfk4 + kj * w.sf_qk, (uint32_t)w.sf_qk, &bars->kv_full[s]);
-            tc::bulk_g2s(st + kStSFV, w.sfv4 + kj * w.sf_v, (uint32_t)w.sf_v, &bars->kv_full[s]);
+          for (int x = 0; x < nx; ++x) {
+            if (t + kPrefetch / 2 < nb)
+              kv_prefetch(bhx[x], list_j(l8x[x], l4x[x], t + kPrefetch / 2), t + kPrefetch / 2 < n8);
+            const int j = list_j(l8x[x], l4x[x], t);
+            const size_t kj = (size_t)bhx[x] * N + j;
+            const uint32_t s = gkv % kStages, ks = gkv / kStages;
+            ++gkv;
+            wait_bar(&bars->kv_empty[s], (ks & 1) ^ 1, w.err);
+            uint8_t* st = sm + kStage0 + s * kStageBytes;
+            if (fp8) {
+              tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * BS * D);
+              tc::bulk_g2s(st + kStK, w.k8 + kj * w.tile8_qk, BS * D, &bars->kv_full[s]);
+              tc::bulk_g2s(st + kStV, w.v8 + kj * w.tile8_v, BS * D, &bars->kv_full[s]);
+            } else {
+              const uint32_t bytes = BS * D / 2 + D * KV4 / 2 + (uint32_t)w.sf_qk + (uint32_t)w.sf_v;
+              tc::mbar_arrive_expect_tx(&bars->kv_full[s], bytes);
+              tc::bulk_g2s(st + kStK, w.k4 + kj * w.tile4_qk, BS * D / 2, &bars->kv_full[s]);
+              tc::bulk_g2s(st + kStV, w.v4 + kj * w.tile4_v, D * KV4 / 2, &bars->kv_full[s]);
+              tc::bulk_g2s(st + kStSFK, w.sfk4 + kj * w.sf_qk, (uint32_t)w.sf_qk, &bars->kv_full[s]);
+              tc::bulk_g2s(st + kStSFV, w.sfv4 + kj * w.sf_v, (uint32_t)w.sf_v, &bars->kv_full[s]);
+            }
           }
         }
       }
     }
   } else if (warp == kMmaWarp) {
     // ===================== MMA issue =====================
-    if (lane == 0) {
+    if (lane == 0 && nb > 0) {
       const uint32_t id8_s = tc::idesc_e4m3(128, BS), id4_s = tc::idesc_nvf4(128, BS);
       const uint32_t id8_o = tc::idesc_e4m3(128, D), id4_o = tc::idesc_nvf4(128, D);
-      uint32_t gblk = 0, wi = 0;
-      for (int item = blockIdx.x; item < total; item += gridDim.x, ++wi) {
-        if (nb == 0) continue;
-        wait_bar(&bars->q_full, wi & 1, w.err);
-        tc::fence_after_sync();
-        if (nb > n8)
-          for (int kb = 0; kb < D / 64; ++kb) tc::cp_sf_atom(tmem + kColSFQ + kb * 4, sm + kSFQ + kb * 512);
-        const uint32_t g0 = gblk;
-        auto issue_s = [&](int t) {
-          const uint32_t gb = g0 + t, s = gb % kStages, b = gb & 1;
-          wait_bar(&bars->kv_full[s], (gb / kStages) & 1, w.err);
-          wait_bar(&bars->s_free[b], ((gb >> 1) & 1) ^ 1, w.err);
+      uint32_t gkv = 0;                 // K/V stages consumed (S issue order)
+      uint32_t gs[2] = {0u, 0u};        // S issued per tile (whole launch)
+      uint32_t gp[2] = {0u, 0u};        // P V issued per tile
+      int last_owner = -1;              // tile whose S sits in the S region
+      uint32_t last_gs = 0;
+      uint32_t stage_of[2][2] = {{0u, 0u}, {0u, 0u}};   // stage each tile's pending P V reads
+      for (int k = 0; k < rounds; ++k) {
+        const int nx = has_tile(k, 1) ? 2 : 1;
+        for (int x = 0; x < nx; ++x) {
+          wait_bar(&bars->tb[x].q_full, k & 1, w.err);
           tc::fence_after_sync();
+          if (nb > n8)
+            for (int kb = 0; kb < D / 64; ++kb)
+              tc::cp_sf_atom(tmem + kColSFQ + 8 * x + kb * 4, sm + x * kQBytes + kSFQ + kb * 512);
+        }
+        auto issue_s = [&](int x, int t) {
+          // the S region is free once its previous owner's softmax has read it
+          if (last_owner >= 0) wait_bar(&bars->tb[last_owner].s_free, last_gs & 1, w.err);
+          const uint32_t s = gkv % kStages;
+          wait_bar(&bars->kv_full[s], (gkv / kStages) & 1, w.err);
+          tc::fence_after_sync();
+          stage_of[x][t & 1] = s;
+          ++gkv;
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
-          const uint32_t dS = tmem + kColS + b * 128;
+          const uint8_t* qs = sm + x * kQBytes;
           if (t < n8) {
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)
-              tc::mma_e4m3(dS, tc::sdesc(sm + kQ8 + kk * 256, 128, D * 8),
+              tc::mma_e4m3(tmem + kColS, tc::sdesc(qs + kQ8 + kk * 256, 128, D * 8),
                            tc::sdesc(st + kStK + kk * 256, 128, D * 8), id8_s, kk > 0);
           } else {
             for (int kb = 0; kb < D / 64; ++kb)
-              tc::cp_sf_atom(tmem + kColSFK + b * 8 + kb * 4, st + kStSFK + kb * 512);
+              tc::cp_sf_atom(tmem + kColSFK + 8 * x + kb * 4, st + kStSFK + kb * 512);
 #pragma unroll
             for (int kk = 0; kk < D / 64; ++kk)
-              tc::mma_nvf4(dS, tc::sdesc(sm + kQ4 + kk * 256, 128, D * 4),
+              tc::mma_nvf4(tmem + kColS, tc::sdesc(qs + kQ4 + kk * 256, 128, D * 4),
                            tc::sdesc(st + kStK + kk * 256, 128, D * 4), id4_s,
-                           tmem + kColSFQ + kk * 4, tmem + kColSFK + b * 8 + kk * 4, kk > 0);
+                           tmem + kColSFQ + 8 * x + kk * 4, tmem + kColSFK + 8 * x + kk * 4, kk > 0);
           }
-          tc::mma_commit(&bars->s_full[b]);
+          tc::mma_commit(&bars->tb[x].s_full);
+          last_owner = x;
+          last_gs = gs[x]++;
         };
-        auto issue_pv = [&](int t) {
-          const uint32_t gb = g0 + t, s = gb % kStages, pb = gb & 1;
-          wait_bar(&bars->p_full[pb], (gb >> 1) & 1, w.err);
-          if (t == 0) wait_bar(&bars->o_free, (wi & 1) ^ 1, w.err);
+        auto issue_pv = [&](int x, int t) {
+          TileBars* tb = &bars->tb[x];
+          wait_bar(&tb->p_full, gp[x] & 1, w.err);
+          if (t == 0 && k > 0) wait_bar(&tb->o_free, (k - 1) & 1, w.err);
           tc::fence_after_sync();
+          const uint32_t s = stage_of[x][t & 1];
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
-          const uint8_t* pbuf = sm + kP0 + pb * kPBytes;
+          const uint8_t* pbuf = sm + kP0 + x * kPBytes;
+          const uint32_t dO = tmem + (x ? kColO1 : kColO0);
           const uint32_t acc0 = t > 0 ? 1u : 0u;
           if (t < n8) {
 #pragma unroll
             for (int kk = 0; kk < BS / 32; ++kk)
-              tc::mma_e4m3(tmem + kColO, tc::sdesc(pbuf + kPData + kk * 256, 128, BS * 8),
+              tc::mma_e4m3(dO, tc::sdesc(pbuf + kPData + kk * 256, 128, BS * 8),
                            tc::sdesc(st + kStV + kk * 256, 128, BS * 8), id8_o, acc0 | (kk > 0));
           } else {
             for (int kb = 0; kb < KV4 / 64; ++kb) {
-              tc::cp_sf_atom(tmem + kColSFP + pb * 8 + kb * 4, pbuf + kPSF + kb * 512);
-              tc::cp_sf_atom(tmem + kColSFV + pb * 8 + kb * 4, st + kStSFV + kb * 512);
+              tc::cp_sf_atom(tmem + kColSFP + 8 * x + kb * 4, pbuf + kPSF + kb * 512);
+              tc::cp_sf_atom(tmem + kColSFV + 8 * x + kb * 4, st + kStSFV + kb * 512);
             }
 #pragma unroll
             for (int kk = 0; kk < KV4 / 64; ++kk)
-              tc::mma_nvf4(tmem + kColO, tc::sdesc(pbuf + kPData + kk * 256, 128, KV4 * 4),
+              tc::mma_nvf4(dO, tc::sdesc(pbuf + kPData + kk * 256, 128, KV4 * 4),
                            tc::sdesc(st + kStV + kk * 256, 128, KV4 * 4), id4_o,
-                           tmem + kColSFP + pb * 8 + kk * 4, tmem + kColSFV + pb * 8 + kk * 4,
+                           tmem + kColSFP + 8 * x + kk * 4, tmem + kColSFV + 8 * x + kk * 4,
                            acc0 | (kk > 0));
           }
-          tc::mma_commit(&bars->p_free[pb]);
+          tc::mma_commit(&tb->p_free);
           tc::mma_commit(&bars->kv_empty[s]);
+          ++gp[x];
         };
-        // S of the first two blocks, then each P V as soon as its P is ready, followed by
-        // the S two blocks ahead (so a late K/V tile never holds back a P V)
-        issue_s(0);
-        if (nb > 1) issue_s(1);
+        issue_s(0, 0);
+        if (nx == 2) issue_s(1, 0);
         for (int t = 0; t < nb; ++t) {
-          issue_pv(t);
-          if (t + 2 < nb) issue_s(t + 2);
+          for (int x = 0; x < nx; ++x) {
+            issue_pv(x, t);
+            if (t + 1 < nb) issue_s(x, t + 1);
+          }
         }
-        tc::mma_commit(&bars->q_empty);
-        tc::mma_commit(&bars->o_full);
-        gblk += nb;
+        for (int x = 0; x < nx; ++x) {
+          tc::mma_commit(&bars->tb[x].q_empty);
+          tc::mma_commit(&bars->tb[x].o_full);
+        }
       }
       tc::mma_commit(&bars->done);
       wait_bar(&bars->done, 0, w.err, false);   // all MMAs retired before TMEM is freed
     }
+  }
   } else {
-    // ===================== softmax + epilogue (warps 0-3) =====================
-    const int r = tid;                                   // query row = TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ============ softmax + epilogue (warps 0-3: tile A, 4-7: tile B) ============
+    const int x = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;               // query row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t colO = x ? kColO1 : kColO0;
+    TileBars* tb = &bars->tb[x];
+    uint8_t* pbuf = sm + kP0 + x * kPBytes;
     const int fpf = g.ny * g.nx;
-    uint32_t gblk = 0, wi = 0;
-    for (int item = blockIdx.x; item < total; item += gridDim.x, ++wi) {
+    uint32_t gx = 0;                                     // blocks of this tile so far
+    for (int k = 0; k < rounds; ++k) {
+      if (!has_tile(k, x)) break;
+      const int item = item_of(k, x);
       const int bh = item / N, i = item - bh * N;
       const size_t qi = (size_t)bh * N + i;
       int hq, wq;
@@ -469,9 +513,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       const int16_t* l8 = w.list8 + qi * w.n8s;
       const int16_t* l4 = w.list4 + qi * w.n4s;
       float m = -INFINITY, l = 0.0f;
-      // block index j, logit scale c and edge geometry of each visited block, fetched two
-      // (list entry) and one (scale) blocks ahead; raw list entries are clamped only
-      // where they are used, so that the loads stay in flight across the block
+      // block index j and logit scale c of each visited block, fetched two (list entry)
+      // and one (scale) blocks ahead; raw list entries are clamped only where they are
+      // used, so that the loads stay in flight across the block
       const float cq = sq * g.sm_scale * kLog2e;
       const float* skh = w.sk + (size_t)bh * N;
       auto list_raw = [&](int t) -> int { return t < n8 ? l8[t] : l4[t - n8]; };
@@ -479,22 +523,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       int j_next = nb > 1 ? list_raw(1) : 0;
       int j_cur = clampj(list_raw(0));
       float sk_cur = skh[j_cur];
-      for (int t = 0; t < nb; ++t, ++gblk) {
+      for (int t = 0; t < nb; ++t, ++gx) {
         const int j_after = t + 2 < nb ? list_raw(t + 2) : 0;
         const int jn = clampj(j_next);
         const float sk_next = skh[jn];
         const int ecls = sm[kEdge + j_cur];
         const float c = cq * sk_cur;
         if (t < n8)
-          softmax_block<D, BS, true>(w, bars, sm, tmem, lane_base, r, c, ecls, gblk, t, m, l);
+          softmax_block<D, BS, true>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
         else
-          softmax_block<D, BS, false>(w, bars, sm, tmem, lane_base, r, c, ecls, gblk, t, m, l);
+          softmax_block<D, BS, false>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
         j_cur = jn;
         sk_cur = sk_next;
         j_next = j_after;
       }
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
-      wait_bar(&bars->o_full, wi & 1, w.err);
+      wait_bar(&tb->o_full, k & 1, w.err);
       tc::fence_after_sync();
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;     // l holds 448 * row sum
       const float* sv = w.sv + (size_t)bh * D;
@@ -502,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       for (int h0 = 0; h0 < D; h0 += 64) {
         uint32_t rr[64];
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColO + h0 + c0, rr + c0);
+        for (int c0 = 0; c0 < 64; c0 += 16) tc::tmem_ld16(tmem + lane_base + colO + h0 + c0, rr + c0);
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 16) tc::tmem_wait_ld16(rr + c0);
         if (row_ok) {
@@ -522,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         }
       }
       tc::fence_before_sync();
-      tc::mbar_arrive(&bars->o_free);
+      tc::mbar_arrive(&tb->o_free);
     }
   }
   tc::fence_before_sync();
