@@ -466,8 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         if (nx == 2) issue_s(1, 0);
         for (int t = 0; t < nb; ++t) {
           for (int x = 0; x < nx; ++x) {
-            issue_pv(x, t);
             if (t + 1 < nb) issue_s(x, t + 1);
+            issue_pv(x, t);
           }
         }
         for (int x = 0; x < nx; ++x) {
