@@ -382,6 +382,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           }
         }
       }
+      // Every copy issued above has landed before this thread leaves (normally they were
+      // consumed long ago; after an aborted wait they may still be in flight).
+      for (uint32_t s = 0; s < (uint32_t)kStages && s < gkv; ++s) {
+        const uint32_t last = s + ((gkv - 1 - s) / kStages) * kStages;
+        wait_bar(&bars->kv_full[s], (last / kStages) & 1, w.err, false);
+      }
+      for (int x = 0; x < 2; ++x) {
+        int kl = -1;
+        for (int k = 0; k < rounds; ++k)
+          if (has_tile(k, x)) kl = k;
+        if (kl >= 0) wait_bar(&bars->tb[x].q_full, kl & 1, w.err, false);
+      }
     }
   } else if (warp == kMmaWarp) {
     // ===================== MMA issue =====================
@@ -466,8 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         if (nx == 2) issue_s(1, 0);
         for (int t = 0; t < nb; ++t) {
           for (int x = 0; x < nx; ++x) {
-            if (t + 1 < nb) issue_s(x, t + 1);
             issue_pv(x, t);
+            if (t + 1 < nb) issue_s(x, t + 1);
           }
         }
         for (int x = 0; x < nx; ++x) {
