@@ -64,6 +64,32 @@ def prep_bytes(w) -> float:
     return float(rd + wr)
 
 
+ATTN_SOURCES = ("attn_tc.cu", "tc.cuh", "common.cuh")
+
+
+def attn_source_hash() -> str:
+    """sha256 over the attention kernel's sources (the DRAM counters belong to one version)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "sparse_mixed_precision_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def attention_traffic(w):
+    """DRAM bytes (read + write) of one attention launch on this workload, from the ncu
+    counters stored in profiles/traffic.json, scaled by (batch x heads) from the captured
+    case; None when there are none or the kernel sources changed since they were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    if rec.get("source_sha256") != attn_source_hash() or rec.get("workload") != w.name:
+        return None
+    return rec["attention_dram_bytes"] * (w.B * w.H) / rec["captured_bh"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -317,10 +343,7 @@ def main():
     peak_eff = (f8 + f4) / (t_roof_attn * 1e-3) / 1e12
     prep_ms = statistics.mean(stage["prepare"])
     pb = prep_bytes(w)
-    traffic_path = os.path.join(ROOT, "profiles", "traffic.json")
-    traffic = None
-    if os.path.exists(traffic_path):
-        traffic = json.load(open(traffic_path)).get("attention_bytes_per_launch")
+    traffic = attention_traffic(w)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
