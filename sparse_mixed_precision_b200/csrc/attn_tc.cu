@@ -29,10 +29,11 @@
 //   warp 9      producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
 //   warps 10-11 idle
 // Tensor memory: O of each tile, ONE S region the two tiles take in turns, and scale
-// factors. MMA order: S_A(0), S_B(0), then per block t: PV_A(t), S_A(t+1), PV_B(t),
-// S_B(t+1); K/V stages are filled and released in that order.
-// Every mbarrier wait is bounded; a wait that runs out sets the workspace error word and
-// the kernel carries on to a clean exit.
+// factors. MMA order: S_A(0), S_B(0), then per block t: S_A(t+1), PV_A(t), S_B(t+1),
+// PV_B(t); K/V stages are filled in S order and released after their P V.
+// Every mbarrier wait is bounded; a wait that runs out sets the workspace error word, each
+// role stops issuing work, the producer waits for its copies in flight and the MMA thread
+// for its MMAs, and the kernel frees its tensor memory and exits.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -133,14 +134,14 @@ __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, in
 // quantised P bytes (E4M3, or E2M1 with an E4M3 scale per 16 keys) stored straight into
 // the tile's P buffer -> O rescale by alpha in TMEM when the max moved (after the tile's
 // previous P V has landed) -> P ready.
-// gx counts this tile's blocks over the whole launch.
+// gx counts this tile's blocks over the whole launch. Returns false when a wait ran out.
 template <int D, int BS, bool FP8>
-__device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t* sm, uint8_t* pbuf,
+__device__ __forceinline__ bool softmax_block(const Ws& w, TileBars* tb, uint8_t* sm, uint8_t* pbuf,
                                               uint32_t tmem, uint32_t lane_base, uint32_t colO, int r,
                                               float c, int ecls, uint32_t gx, int t, float& m, float& l) {
   constexpr int NG = BS / 16;
   constexpr int KV4 = BS < 64 ? 64 : BS;
-  wait_bar(&tb->s_full, gx & 1, w.err);
+  if (!wait_bar(&tb->s_full, gx & 1, w.err)) return false;
   tc::fence_after_sync();
   uint32_t sr[BS];
 #pragma unroll
@@ -176,7 +177,7 @@ __device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t
   const float bias = kLog2_448 - m_new;
   // the P buffer (and O) are free once this tile's previous P V has completed
   if (t > 0) {
-    wait_bar(&tb->p_free, (gx - 1) & 1, w.err);
+    if (!wait_bar(&tb->p_free, (gx - 1) & 1, w.err)) return false;
     tc::fence_after_sync();
   }
   float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -245,6 +246,7 @@ __device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t
   tc::fence_proxy_async_smem();
   tc::fence_before_sync();
   tc::mbar_arrive(&tb->p_full);
+  return true;
 }
 
 template <int D, int BS>
@@ -333,12 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           tc::prefetch_l2(w.v4 + kj * w.tile4_v, D * KV4 / 2);
         }
       };
-      for (int k = 0; k < rounds; ++k) {
+      bool dead = false;                // a wait ran out: issue nothing more
+      int q_rounds[2] = {0, 0};         // Q tiles loaded per tile
+      for (int k = 0; k < rounds && !dead; ++k) {
         const int nx = has_tile(k, 1) ? 2 : 1;
         int bhx[2], ix[2];
         const int16_t* l8x[2];
         const int16_t* l4x[2];
-        for (int x = 0; x < nx; ++x) {
+        for (int x = 0; x < nx && !dead; ++x) {
           const int item = item_of(k, x);
           bhx[x] = item / N;
           ix[x] = item - bhx[x] * N;
@@ -346,17 +350,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           l8x[x] = w.list8 + qi * w.n8s;
           l4x[x] = w.list4 + qi * w.n4s;
           TileBars* tb = &bars->tb[x];
-          wait_bar(&tb->q_empty, (k & 1) ^ 1, w.err);
+          if (!wait_bar(&tb->q_empty, (k & 1) ^ 1, w.err)) { dead = true; break; }
           const uint32_t qbytes = BS * D + BS * D / 2 + (uint32_t)w.sf_qk;
           uint8_t* qs = sm + x * kQBytes;
           tc::mbar_arrive_expect_tx(&tb->q_full, qbytes);
           tc::bulk_g2s(qs + kQ8, w.q8 + qi * w.tile8_qk, BS * D, &tb->q_full);
           tc::bulk_g2s(qs + kQ4, w.q4 + qi * w.tile4_qk, BS * D / 2, &tb->q_full);
           tc::bulk_g2s(qs + kSFQ, w.sfq4 + qi * w.sf_qk, (uint32_t)w.sf_qk, &tb->q_full);
+          ++q_rounds[x];
         }
+        if (dead) break;
         for (int t = 0; t < kPrefetch / 2 && t < nb; ++t)
           for (int x = 0; x < nx; ++x) kv_prefetch(bhx[x], list_j(l8x[x], l4x[x], t), t < n8);
-        for (int t = 0; t < nb; ++t) {
+        for (int t = 0; t < nb && !dead; ++t) {
           const bool fp8 = t < n8;
           for (int x = 0; x < nx; ++x) {
             if (t + kPrefetch / 2 < nb)
@@ -364,8 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
             const int j = list_j(l8x[x], l4x[x], t);
             const size_t kj = (size_t)bhx[x] * N + j;
             const uint32_t s = gkv % kStages, ks = gkv / kStages;
-            ++gkv;
-            wait_bar(&bars->kv_empty[s], (ks & 1) ^ 1, w.err);
+            if (!wait_bar(&bars->kv_empty[s], (ks & 1) ^ 1, w.err)) { dead = true; break; }
             uint8_t* st = sm + kStage0 + s * kStageBytes;
             if (fp8) {
               tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * BS * D);
@@ -379,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
               tc::bulk_g2s(st + kStSFK, w.sfk4 + kj * w.sf_qk, (uint32_t)w.sf_qk, &bars->kv_full[s]);
               tc::bulk_g2s(st + kStSFV, w.sfv4 + kj * w.sf_v, (uint32_t)w.sf_v, &bars->kv_full[s]);
             }
+            ++gkv;
           }
         }
       }
@@ -388,40 +394,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         const uint32_t last = s + ((gkv - 1 - s) / kStages) * kStages;
         wait_bar(&bars->kv_full[s], (last / kStages) & 1, w.err, false);
       }
-      for (int x = 0; x < 2; ++x) {
-        int kl = -1;
-        for (int k = 0; k < rounds; ++k)
-          if (has_tile(k, x)) kl = k;
-        if (kl >= 0) wait_bar(&bars->tb[x].q_full, kl & 1, w.err, false);
-      }
+      for (int x = 0; x < 2; ++x)
+        if (q_rounds[x] > 0) wait_bar(&bars->tb[x].q_full, (q_rounds[x] - 1) & 1, w.err, false);
     }
   } else if (warp == kMmaWarp) {
     // ===================== MMA issue =====================
     if (lane == 0 && nb > 0) {
       const uint32_t id8_s = tc::idesc_e4m3(128, BS), id4_s = tc::idesc_nvf4(128, BS);
       const uint32_t id8_o = tc::idesc_e4m3(128, D), id4_o = tc::idesc_nvf4(128, D);
-      uint32_t gkv = 0;                 // K/V stages consumed (S issue order)
-      uint32_t gs[2] = {0u, 0u};        // S issued per tile (whole launch)
-      uint32_t gp[2] = {0u, 0u};        // P V issued per tile
-      int last_owner = -1;              // tile whose S sits in the S region
+      uint32_t gkv = 0;                 // K/V stages consumed (S issue order: A0 B0 A1 B1 ...)
+      int last_owner = -1;              // tile whose S sits in the S region, and its block index
       uint32_t last_gs = 0;
-      uint32_t stage_of[2][2] = {{0u, 0u}, {0u, 0u}};   // stage each tile's pending P V reads
-      for (int k = 0; k < rounds; ++k) {
+      bool dead = false;                // a wait ran out: issue nothing more
+      for (int k = 0; k < rounds && !dead; ++k) {
         const int nx = has_tile(k, 1) ? 2 : 1;
-        for (int x = 0; x < nx; ++x) {
-          wait_bar(&bars->tb[x].q_full, k & 1, w.err);
+        const uint32_t gbase = (uint32_t)k * (uint32_t)nb;   // blocks each tile had in earlier rounds
+        const uint32_t kvbase = gkv;                          // stage sequence number of S_A(0)
+        for (int x = 0; x < nx && !dead; ++x) {
+          dead = !wait_bar(&bars->tb[x].q_full, k & 1, w.err);
           tc::fence_after_sync();
-          if (nb > n8)
+          if (!dead && nb > n8)
             for (int kb = 0; kb < D / 64; ++kb)
               tc::cp_sf_atom(tmem + kColSFQ + 8 * x + kb * 4, sm + x * kQBytes + kSFQ + kb * 512);
         }
-        auto issue_s = [&](int x, int t) {
+        // S = Q K^T of tile x for its block t, into the shared S region
+        auto issue_s = [&](int x, int t) -> bool {
           // the S region is free once its previous owner's softmax has read it
-          if (last_owner >= 0) wait_bar(&bars->tb[last_owner].s_free, last_gs & 1, w.err);
+          if (last_owner >= 0 && !wait_bar(&bars->tb[last_owner].s_free, last_gs & 1, w.err)) return false;
           const uint32_t s = gkv % kStages;
-          wait_bar(&bars->kv_full[s], (gkv / kStages) & 1, w.err);
+          if (!wait_bar(&bars->kv_full[s], (gkv / kStages) & 1, w.err)) return false;
           tc::fence_after_sync();
-          stage_of[x][t & 1] = s;
           ++gkv;
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
           const uint8_t* qs = sm + x * kQBytes;
@@ -441,14 +443,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           }
           tc::mma_commit(&bars->tb[x].s_full);
           last_owner = x;
-          last_gs = gs[x]++;
+          last_gs = gbase + (uint32_t)t;
+          return true;
         };
-        auto issue_pv = [&](int x, int t) {
+        // O += P V of tile x for its block t; its K/V stage is the S issue sequence number
+        // kvbase + nx t + x modulo the ring size
+        auto issue_pv = [&](int x, int t) -> bool {
           TileBars* tb = &bars->tb[x];
-          wait_bar(&tb->p_full, gp[x] & 1, w.err);
-          if (t == 0 && k > 0) wait_bar(&tb->o_free, (k - 1) & 1, w.err);
+          if (!wait_bar(&tb->p_full, (gbase + (uint32_t)t) & 1, w.err)) return false;
+          if (t == 0 && k > 0 && !wait_bar(&tb->o_free, (k - 1) & 1, w.err)) return false;
           tc::fence_after_sync();
-          const uint32_t s = stage_of[x][t & 1];
+          const uint32_t s = (kvbase + (uint32_t)(nx * t + x)) % kStages;
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
           const uint8_t* pbuf = sm + kP0 + x * kPBytes;
           const uint32_t dO = tmem + (x ? kColO1 : kColO0);
@@ -472,20 +477,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           }
           tc::mma_commit(&tb->p_free);
           tc::mma_commit(&bars->kv_empty[s]);
-          ++gp[x];
+          return true;
         };
-        issue_s(0, 0);
-        if (nx == 2) issue_s(1, 0);
-        for (int t = 0; t < nb; ++t) {
-          for (int x = 0; x < nx; ++x) {
-            issue_pv(x, t);
-            if (t + 1 < nb) issue_s(x, t + 1);
+        // A tile's next S goes into the S region as soon as the other tile has read its own
+        // S (or, alone, as soon as this tile has), so that it is ready when this tile's
+        // softmax finishes the current block; the P V follows once that block's P is stored.
+        if (!dead) dead = !issue_s(0, 0);
+        if (!dead && nx == 2) dead = !issue_s(1, 0);
+        for (int t = 0; t < nb && !dead; ++t)
+          for (int x = 0; x < nx && !dead; ++x) {
+            if (t + 1 < nb) dead = !issue_s(x, t + 1);
+            if (!dead) dead = !issue_pv(x, t);
           }
-        }
-        for (int x = 0; x < nx; ++x) {
-          tc::mma_commit(&bars->tb[x].q_empty);
-          tc::mma_commit(&bars->tb[x].o_full);
-        }
+        if (!dead)
+          for (int x = 0; x < nx; ++x) {
+            tc::mma_commit(&bars->tb[x].q_empty);
+            tc::mma_commit(&bars->tb[x].o_full);
+          }
       }
       tc::mma_commit(&bars->done);
       wait_bar(&bars->done, 0, w.err, false);   // all MMAs retired before TMEM is freed
@@ -501,7 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
     uint8_t* pbuf = sm + kP0 + x * kPBytes;
     const int fpf = g.ny * g.nx;
     uint32_t gx = 0;                                     // blocks of this tile so far
-    for (int k = 0; k < rounds; ++k) {
+    bool dead = false;                                   // a wait ran out: stop
+    for (int k = 0; k < rounds && !dead; ++k) {
       if (!has_tile(k, x)) break;
       const int item = item_of(k, x);
       const int bh = item / N, i = item - bh * N;
@@ -541,16 +550,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         const float sk_next = skh[jn];
         const int ecls = sm[kEdge + j_cur];
         const float c = cq * sk_cur;
-        if (t < n8)
-          softmax_block<D, BS, true>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
-        else
-          softmax_block<D, BS, false>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
+        const bool ok =
+            t < n8 ? softmax_block<D, BS, true>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l)
+                   : softmax_block<D, BS, false>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
+        if (!ok) {
+          dead = true;
+          break;
+        }
         j_cur = jn;
         sk_cur = sk_next;
         j_next = j_after;
       }
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
-      wait_bar(&tb->o_full, k & 1, w.err);
+      if (dead || !wait_bar(&tb->o_full, k & 1, w.err)) {
+        dead = true;
+        break;
+      }
       tc::fence_after_sync();
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;     // l holds 448 * row sum
       const float* sv = w.sv + (size_t)bh * D;
