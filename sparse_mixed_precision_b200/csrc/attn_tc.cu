@@ -134,14 +134,17 @@ __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, in
 // quantised P bytes (E4M3, or E2M1 with an E4M3 scale per 16 keys) stored straight into
 // the tile's P buffer -> O rescale by alpha in TMEM when the max moved (after the tile's
 // previous P V has landed) -> P ready.
-// gx counts this tile's blocks over the whole launch. Returns false when a wait ran out.
+// gx counts this tile's blocks over the whole launch. A wait that runs out does not stop
+// the block (checking here costs the loop several percent): after a timeout every later
+// wait returns at once, so the rest of the round runs through without waiting and the
+// warpgroup stops at the round's epilogue.
 template <int D, int BS, bool FP8>
-__device__ __forceinline__ bool softmax_block(const Ws& w, TileBars* tb, uint8_t* sm, uint8_t* pbuf,
+__device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t* sm, uint8_t* pbuf,
                                               uint32_t tmem, uint32_t lane_base, uint32_t colO, int r,
                                               float c, int ecls, uint32_t gx, int t, float& m, float& l) {
   constexpr int NG = BS / 16;
   constexpr int KV4 = BS < 64 ? 64 : BS;
-  if (!wait_bar(&tb->s_full, gx & 1, w.err)) return false;
+  wait_bar(&tb->s_full, gx & 1, w.err);
   tc::fence_after_sync();
   uint32_t sr[BS];
 #pragma unroll
@@ -177,7 +180,7 @@ __device__ __forceinline__ bool softmax_block(const Ws& w, TileBars* tb, uint8_t
   const float bias = kLog2_448 - m_new;
   // the P buffer (and O) are free once this tile's previous P V has completed
   if (t > 0) {
-    if (!wait_bar(&tb->p_free, (gx - 1) & 1, w.err)) return false;
+    wait_bar(&tb->p_free, (gx - 1) & 1, w.err);
     tc::fence_after_sync();
   }
   float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -246,7 +249,6 @@ __device__ __forceinline__ bool softmax_block(const Ws& w, TileBars* tb, uint8_t
   tc::fence_proxy_async_smem();
   tc::fence_before_sync();
   tc::mbar_arrive(&tb->p_full);
-  return true;
 }
 
 template <int D, int BS>
@@ -550,19 +552,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         const float sk_next = skh[jn];
         const int ecls = sm[kEdge + j_cur];
         const float c = cq * sk_cur;
-        const bool ok =
-            t < n8 ? softmax_block<D, BS, true>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l)
-                   : softmax_block<D, BS, false>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
-        if (!ok) {
-          dead = true;
-          break;
-        }
+        if (t < n8)
+          softmax_block<D, BS, true>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
+        else
+          softmax_block<D, BS, false>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
         j_cur = jn;
         sk_cur = sk_next;
         j_next = j_after;
       }
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
-      if (dead || !wait_bar(&tb->o_full, k & 1, w.err)) {
+      if (!wait_bar(&tb->o_full, k & 1, w.err)) {
         dead = true;
         break;
       }
