@@ -536,29 +536,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       const int16_t* l8 = w.list8 + qi * w.n8s;
       const int16_t* l4 = w.list4 + qi * w.n4s;
       float m = -INFINITY, l = 0.0f;
-      // block index j and logit scale c of each visited block, fetched two (list entry)
-      // and one (scale) blocks ahead; raw list entries are clamped only where they are
-      // used, so that the loads stay in flight across the block
+      // Block index j and key scale s_k[j] of every visited block, fetched 32 blocks at a
+      // time (lane i holds block 32 ch + i) and broadcast by shuffles: the list entries of
+      // chunk ch + 2 and the scales of chunk ch + 1 are loaded at the start of chunk ch,
+      // so no block waits on a global load.
       const float cq = sq * g.sm_scale * kLog2e;
       const float* skh = w.sk + (size_t)bh * N;
-      auto list_raw = [&](int t) -> int { return t < n8 ? l8[t] : l4[t - n8]; };
-      auto clampj = [&](int j) -> int { return (j < 0 || j >= N) ? 0 : j; };
-      int j_next = nb > 1 ? list_raw(1) : 0;
-      int j_cur = clampj(list_raw(0));
-      float sk_cur = skh[j_cur];
+      auto list_j = [&](int t) -> int {
+        const int j = t < nb ? (t < n8 ? l8[t] : l4[t - n8]) : 0;
+        return (j < 0 || j >= N) ? 0 : j;
+      };
+      int jA = list_j(lane), jB = list_j(32 + lane), jC = list_j(64 + lane);
+      float sA = skh[jA], sB = skh[jB];
       for (int t = 0; t < nb; ++t, ++gx) {
-        const int j_after = t + 2 < nb ? list_raw(t + 2) : 0;
-        const int jn = clampj(j_next);
-        const float sk_next = skh[jn];
-        const int ecls = sm[kEdge + j_cur];
-        const float c = cq * sk_cur;
+        const int ln = t & 31;
+        const int j = __shfl_sync(0xffffffffu, jA, ln);
+        const float c = cq * __shfl_sync(0xffffffffu, sA, ln);
+        if (ln == 31) {                                   // next chunk
+          jA = jB;
+          sA = sB;
+          jB = jC;
+          sB = skh[jB];
+          jC = list_j(t + 65 + lane);
+        }
+        const int ecls = sm[kEdge + j];
         if (t < n8)
           softmax_block<D, BS, true>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
         else
           softmax_block<D, BS, false>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
-        j_cur = jn;
-        sk_cur = sk_next;
-        j_next = j_after;
       }
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
       if (!wait_bar(&tb->o_full, k & 1, w.err)) {
