@@ -25,12 +25,15 @@
 // L2); round k of a CTA takes its work items 2k (tile A) and 2k+1 (tile B):
 //   warps 0-3   softmax + epilogue of tile A: thread r owns query row r (TMEM lane r)
 //   warps 4-7   softmax + epilogue of tile B
-//   warp 8      MMA issue (one thread) and TMEM allocation
+//   warp 8      MMA issue for tile A (one thread) and TMEM allocation
 //   warp 9      producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
-//   warps 10-11 idle
+//   warp 10     MMA issue for tile B (one thread)
+//   warp 11     idle
 // Tensor memory: O of each tile, ONE S region the two tiles take in turns, and scale
-// factors. MMA order: S_A(0), S_B(0), then per block t: S_A(t+1), PV_A(t), S_B(t+1),
-// PV_B(t); K/V stages are filled in S order and released after their P V.
+// factors. Each tile's issuer runs S(0), then per block t: S(t+1), PV(t); the S region is
+// taken in the order S_A(t), S_B(t), S_A(t+1), ..., each S waiting until the softmax of
+// the previous owner has read its own. K/V stages are filled in that S order and released
+// after their P V.
 // Every mbarrier wait is bounded; a wait that runs out sets the workspace error word, each
 // role stops issuing work, the producer waits for its copies in flight and the MMA thread
 // for its MMAs, and the kernel frees its tensor memory and exits.
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       tc::mbar_init(&tb->o_full, 1);
       tc::mbar_init(&tb->o_free, 128);
     }
-    tc::mbar_init(&bars->done, 1);
+    tc::mbar_init(&bars->done, 2);
     tc::fence_mbar_init();
   }
   for (uint32_t o = tid * 16; o < kStage0; o += kThreads * 16)
@@ -399,36 +402,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       for (int x = 0; x < 2; ++x)
         if (q_rounds[x] > 0) wait_bar(&bars->tb[x].q_full, (q_rounds[x] - 1) & 1, w.err, false);
     }
-  } else if (warp == kMmaWarp) {
-    // ===================== MMA issue =====================
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 2) {
+    // ============ MMA issue: one thread per tile (warp 8: tile A, warp 10: tile B) ============
+    const int x = warp == kMmaWarp ? 0 : 1;
     if (lane == 0 && nb > 0) {
       const uint32_t id8_s = tc::idesc_e4m3(128, BS), id4_s = tc::idesc_nvf4(128, BS);
       const uint32_t id8_o = tc::idesc_e4m3(128, D), id4_o = tc::idesc_nvf4(128, D);
-      uint32_t gkv = 0;                 // K/V stages consumed (S issue order: A0 B0 A1 B1 ...)
-      int last_owner = -1;              // tile whose S sits in the S region, and its block index
-      uint32_t last_gs = 0;
+      TileBars* tb = &bars->tb[x];
+      const uint8_t* qs = sm + x * kQBytes;
+      const uint8_t* pbuf = sm + kP0 + x * kPBytes;
+      const uint32_t dO = tmem + (x ? kColO1 : kColO0);
       bool dead = false;                // a wait ran out: issue nothing more
       for (int k = 0; k < rounds && !dead; ++k) {
+        if (!has_tile(k, x)) break;     // only tile B can be missing, in the last round only
         const int nx = has_tile(k, 1) ? 2 : 1;
         const uint32_t gbase = (uint32_t)k * (uint32_t)nb;   // blocks each tile had in earlier rounds
-        const uint32_t kvbase = gkv;                          // stage sequence number of S_A(0)
-        for (int x = 0; x < nx && !dead; ++x) {
-          dead = !wait_bar(&bars->tb[x].q_full, k & 1, w.err);
+        const uint32_t kvbase = 2u * gbase;                  // K/V stages of earlier rounds (2 tiles each)
+        dead = !wait_bar(&tb->q_full, k & 1, w.err);
+        tc::fence_after_sync();
+        if (!dead && nb > n8)
+          for (int kb = 0; kb < D / 64; ++kb)
+            tc::cp_sf_atom(tmem + kColSFQ + 8 * x + kb * 4, qs + kSFQ + kb * 512);
+        // The S region is taken in the order A0 B0 A1 B1 ... (A0 A1 ... when B is absent),
+        // continuing across rounds; S of this tile's block t waits until the softmax of the
+        // previous owner has read its S.
+        auto issue_s = [&](int t) -> bool {
+          if (x == 1) {
+            if (!wait_bar(&bars->tb[0].s_free, (gbase + t) & 1, w.err)) return false;
+          } else if (t > 0) {
+            if (!wait_bar(&bars->tb[nx - 1].s_free, (gbase + t - 1) & 1, w.err)) return false;
+          } else if (k > 0) {
+            if (!wait_bar(&bars->tb[1].s_free, (gbase - 1) & 1, w.err)) return false;
+          }
+          const uint32_t seq = kvbase + (uint32_t)(nx * t + x);   // K/V stage sequence number
+          const uint32_t s = seq % kStages;
+          if (!wait_bar(&bars->kv_full[s], (seq / kStages) & 1, w.err)) return false;
           tc::fence_after_sync();
-          if (!dead && nb > n8)
-            for (int kb = 0; kb < D / 64; ++kb)
-              tc::cp_sf_atom(tmem + kColSFQ + 8 * x + kb * 4, sm + x * kQBytes + kSFQ + kb * 512);
-        }
-        // S = Q K^T of tile x for its block t, into the shared S region
-        auto issue_s = [&](int x, int t) -> bool {
-          // the S region is free once its previous owner's softmax has read it
-          if (last_owner >= 0 && !wait_bar(&bars->tb[last_owner].s_free, last_gs & 1, w.err)) return false;
-          const uint32_t s = gkv % kStages;
-          if (!wait_bar(&bars->kv_full[s], (gkv / kStages) & 1, w.err)) return false;
-          tc::fence_after_sync();
-          ++gkv;
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
-          const uint8_t* qs = sm + x * kQBytes;
           if (t < n8) {
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)
@@ -443,22 +453,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
                            tc::sdesc(st + kStK + kk * 256, 128, D * 4), id4_s,
                            tmem + kColSFQ + 8 * x + kk * 4, tmem + kColSFK + 8 * x + kk * 4, kk > 0);
           }
-          tc::mma_commit(&bars->tb[x].s_full);
-          last_owner = x;
-          last_gs = gbase + (uint32_t)t;
+          tc::mma_commit(&tb->s_full);
           return true;
         };
-        // O += P V of tile x for its block t; its K/V stage is the S issue sequence number
-        // kvbase + nx t + x modulo the ring size
-        auto issue_pv = [&](int x, int t) -> bool {
-          TileBars* tb = &bars->tb[x];
+        // O += P V of this tile's block t
+        auto issue_pv = [&](int t) -> bool {
           if (!wait_bar(&tb->p_full, (gbase + (uint32_t)t) & 1, w.err)) return false;
           if (t == 0 && k > 0 && !wait_bar(&tb->o_free, (k - 1) & 1, w.err)) return false;
           tc::fence_after_sync();
           const uint32_t s = (kvbase + (uint32_t)(nx * t + x)) % kStages;
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
-          const uint8_t* pbuf = sm + kP0 + x * kPBytes;
-          const uint32_t dO = tmem + (x ? kColO1 : kColO0);
           const uint32_t acc0 = t > 0 ? 1u : 0u;
           if (t < n8) {
 #pragma unroll
@@ -481,24 +485,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           tc::mma_commit(&bars->kv_empty[s]);
           return true;
         };
-        // A tile's next S goes into the S region as soon as the other tile has read its own
-        // S (or, alone, as soon as this tile has), so that it is ready when this tile's
-        // softmax finishes the current block; the P V follows once that block's P is stored.
-        if (!dead) dead = !issue_s(0, 0);
-        if (!dead && nx == 2) dead = !issue_s(1, 0);
-        for (int t = 0; t < nb && !dead; ++t)
-          for (int x = 0; x < nx && !dead; ++x) {
-            if (t + 1 < nb) dead = !issue_s(x, t + 1);
-            if (!dead) dead = !issue_pv(x, t);
-          }
-        if (!dead)
-          for (int x = 0; x < nx; ++x) {
-            tc::mma_commit(&bars->tb[x].q_empty);
-            tc::mma_commit(&bars->tb[x].o_full);
-          }
+        // This tile's next S is issued as soon as the S region comes free, ahead of the
+        // current block's P V, so that it is ready when the softmax finishes the block.
+        dead = dead || !issue_s(0);
+        for (int t = 0; t < nb && !dead; ++t) {
+          if (t + 1 < nb) dead = !issue_s(t + 1);
+          if (!dead) dead = !issue_pv(t);
+        }
+        if (!dead) {
+          tc::mma_commit(&tb->q_empty);
+          tc::mma_commit(&tb->o_full);
+        }
       }
       tc::mma_commit(&bars->done);
-      wait_bar(&bars->done, 0, w.err, false);   // all MMAs retired before TMEM is freed
+      wait_bar(&bars->done, 0, w.err, false);   // both issuers' MMAs retired before TMEM is freed
     }
   }
   } else {
