@@ -207,22 +207,27 @@ __device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t
     uint32_t sfw[KV4 / 64];
 #pragma unroll
     for (int q = 0; q < KV4 / 64; ++q) sfw[q] = 0u;
+    // group scales first (independent chains): sigma = E4M3(448 p_max / 6), p_max from
+    // the group max
+    float rs[NG];
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
-      // group scale from the group max: sigma = E4M3(448 p_max / 6)
-      uint32_t sc = f32_to_e4m3(ex2(fmaf(gm[q], c, bias)) * (1.0f / 6.0f));
+      const uint32_t sc = f32_to_e4m3(ex2(fmaf(gm[q], c, bias)) * (1.0f / 6.0f));
       const float sg = e4m3_to_f32((uint8_t)sc);
-      const float rs = sg > 0.0f ? rcp_approx(sg) : 0.0f;
+      rs[q] = sg > 0.0f ? rcp_approx(sg) : 0.0f;
+      sfw[q >> 2] |= sc << (8 * (q & 3));
+    }
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
       float y[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const float p = ex2(fmaf(s[16 * q + e], c, bias));
         sum4[e & 3] += p;
-        y[e] = p * rs;
+        y[e] = p * rs[q];
       }
       *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, 8 * q, KV4 / 2)) =
           make_uint2(f32x8_to_e2m1x8(y), f32x8_to_e2m1x8(y + 8));
-      sfw[q >> 2] |= sc << (8 * (q & 3));
     }
 #pragma unroll
     for (int gk = BS; gk < KV4; gk += 16)                  // zero keys past the block (32-token blocks)
