@@ -131,6 +131,25 @@ __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, in
   return hv * wv;
 }
 
+// O row *= alpha in TMEM (D columns from taddr). Out of line: after the first few blocks
+// the running max rarely moves, and the unrolled body would sit in the hot loop's code.
+template <int D>
+__device__ __noinline__ void rescale_o(uint32_t taddr, float alpha) {
+#pragma unroll
+  for (int h0 = 0; h0 < D; h0 += 32) {
+    uint32_t orr[32];
+    tc::tmem_ld16(taddr + h0, orr);
+    tc::tmem_ld16(taddr + h0 + 16, orr + 16);
+    tc::tmem_wait_ld16(orr);
+    tc::tmem_wait_ld16(orr + 16);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+    tc::tmem_st16(taddr + h0, orr);
+    tc::tmem_st16(taddr + h0 + 16, orr + 16);
+  }
+  tc::tmem_wait_st();
+}
+
 // One KV block of one query row of a tile (softmax warps). The S row is read once from
 // the shared S region (which is released at once) -> group maxima -> row max -> alpha ->
 // one fused loop computing p448 = 2^(S c + log2 448 - m_new), the row sum and the
@@ -238,21 +257,7 @@ __device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t
   }
   l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
   // O row *= alpha (the previous P V of this tile has landed: waited above)
-  if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-    for (int h0 = 0; h0 < D; h0 += 32) {
-      uint32_t orr[32];
-      tc::tmem_ld16(tmem + lane_base + colO + h0, orr);
-      tc::tmem_ld16(tmem + lane_base + colO + h0 + 16, orr + 16);
-      tc::tmem_wait_ld16(orr);
-      tc::tmem_wait_ld16(orr + 16);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-      tc::tmem_st16(tmem + lane_base + colO + h0, orr);
-      tc::tmem_st16(tmem + lane_base + colO + h0 + 16, orr + 16);
-    }
-    tc::tmem_wait_st();
-  }
+  if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) rescale_o<D>(tmem + lane_base + colO, alpha);
   m = m_new;
   tc::fence_proxy_async_smem();
   tc::fence_before_sync();
