@@ -67,17 +67,18 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-// TMEM columns (512 allocated): O of tile A and B, the shared S region, scale factors.
+// TMEM columns (512 allocated): O of tile A and B, the shared S region, scale factors,
+// and each tile's quantised P (row r in lane r, 4 bytes of consecutive keys per column;
+// the A operand of its P V MMAs).
 constexpr uint32_t kColO0 = 0, kColO1 = 128, kColS = 256;
 constexpr uint32_t kColSFQ = 384, kColSFK = 400, kColSFP = 416, kColSFV = 432;   // + 8 * tile
+constexpr uint32_t kColP = 448;                                                   // + 32 * tile
 
 // shared memory carve-up (bytes)
 constexpr uint32_t kQ8 = 0, kQ4 = 16384, kSFQ = 24576, kQBytes = 25600;   // per tile
 constexpr uint32_t kStage0 = 2 * kQBytes;
 constexpr uint32_t kStK = 0, kStV = 16384, kStSFK = 32768, kStSFV = 33792, kStageBytes = 34816;
-constexpr uint32_t kP0 = kStage0 + kStages * kStageBytes;
-constexpr uint32_t kPData = 0, kPSF = 16384, kPBytes = 17408;                 // per tile
-constexpr uint32_t kMask = kP0 + 2 * kPBytes;      // 4 slot-validity masks x 4 words
+constexpr uint32_t kMask = kStage0 + kStages * kStageBytes;   // 4 slot-validity masks x 4 words
 constexpr uint32_t kEdge = kMask + 64;             // edge class of every block (u8 [N <= 4096])
 constexpr uint32_t kBar = kEdge + 4096;
 constexpr uint32_t kSmemBytes = kBar + 256;
@@ -160,8 +161,8 @@ __device__ __noinline__ void rescale_o(uint32_t taddr, float alpha) {
 // the block (checking here costs the loop several percent): after a timeout every later
 // wait returns at once, so the rest of the round runs through without waiting and the
 // warpgroup stops at the round's epilogue.
-template <int D, int BS, bool FP8>
-__device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t* sm, uint8_t* pbuf,
+template <int D, int BS>
+__device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileBars* tb, uint8_t* sm, uint32_t colP,
                                               uint32_t tmem, uint32_t lane_base, uint32_t colO, int r,
                                               float c, int ecls, uint32_t gx, int t, float& m, float& l) {
   constexpr int NG = BS / 16;
@@ -220,7 +221,7 @@ __device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t
         }
         wd[e / 4] = (uint32_t)f32x2_to_e4m3x2(p[0], p[1]) | ((uint32_t)f32x2_to_e4m3x2(p[2], p[3]) << 16);
       }
-      *reinterpret_cast<uint4*>(pbuf + kPData + kmajor_off(r, 16 * q, BS)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      tc::tmem_st4(tmem + lane_base + colP + 4 * q, wd);
     }
   } else {
     uint32_t sfw[KV4 / 64];
@@ -245,21 +246,23 @@ __device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t
         sum4[e & 3] += p;
         y[e] = p * rs[q];
       }
-      *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, 8 * q, KV4 / 2)) =
-          make_uint2(f32x8_to_e2m1x8(y), f32x8_to_e2m1x8(y + 8));
+      tc::tmem_st2(tmem + lane_base + colP + 2 * q, f32x8_to_e2m1x8(y), f32x8_to_e2m1x8(y + 8));
     }
 #pragma unroll
     for (int gk = BS; gk < KV4; gk += 16)                  // zero keys past the block (32-token blocks)
-      *reinterpret_cast<uint2*>(pbuf + kPData + kmajor_off(r, gk / 2, KV4 / 2)) = make_uint2(0u, 0u);
+      tc::tmem_st2(tmem + lane_base + colP + gk / 8, 0u, 0u);
+    // This row's scale word for each 64-key step, where the MMA reads it: lane r, column
+    // 4 kb + (r / 32) of the tile's P scale columns (the layout that copying a replicated
+    // 32-row scale atom leaves there).
+    const uint32_t sfp = kColSFP + (colP - kColP) / 4;   // + 8 * tile
 #pragma unroll
-    for (int q = 0; q < KV4 / 64; ++q)
-      *reinterpret_cast<uint32_t*>(pbuf + kPSF + q * 512 + (r & 31) * 16 + (r >> 5) * 4) = sfw[q];
+    for (int q = 0; q < KV4 / 64; ++q) tc::tmem_st1(tmem + lane_base + sfp + 4 * q + (r >> 5), sfw[q]);
   }
   l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
   // O row *= alpha (the previous P V of this tile has landed: waited above)
   if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) rescale_o<D>(tmem + lane_base + colO, alpha);
   m = m_new;
-  tc::fence_proxy_async_smem();
+  tc::tmem_wait_st();                                     // P and its scales are in TMEM
   tc::fence_before_sync();
   tc::mbar_arrive(&tb->p_full);
 }
@@ -420,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       const uint32_t id8_o = tc::idesc_e4m3(128, D), id4_o = tc::idesc_nvf4(128, D);
       TileBars* tb = &bars->tb[x];
       const uint8_t* qs = sm + x * kQBytes;
-      const uint8_t* pbuf = sm + kP0 + x * kPBytes;
+      const uint32_t aP = tmem + kColP + 32 * x;          // P: the A operand of P V, in TMEM
       const uint32_t dO = tmem + (x ? kColO1 : kColO0);
       bool dead = false;                // a wait ran out: issue nothing more
       for (int k = 0; k < rounds && !dead; ++k) {
@@ -477,19 +480,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           if (t < n8) {
 #pragma unroll
             for (int kk = 0; kk < BS / 32; ++kk)
-              tc::mma_e4m3(dO, tc::sdesc(pbuf + kPData + kk * 256, 128, BS * 8),
-                           tc::sdesc(st + kStV + kk * 256, 128, BS * 8), id8_o, acc0 | (kk > 0));
+              tc::mma_e4m3_ta(dO, aP + kk * 8, tc::sdesc(st + kStV + kk * 256, 128, BS * 8), id8_o,
+                              acc0 | (kk > 0));
           } else {
-            for (int kb = 0; kb < KV4 / 64; ++kb) {
-              tc::cp_sf_atom(tmem + kColSFP + 8 * x + kb * 4, pbuf + kPSF + kb * 512);
+            for (int kb = 0; kb < KV4 / 64; ++kb)
               tc::cp_sf_atom(tmem + kColSFV + 8 * x + kb * 4, st + kStSFV + kb * 512);
-            }
 #pragma unroll
             for (int kk = 0; kk < KV4 / 64; ++kk)
-              tc::mma_nvf4(dO, tc::sdesc(pbuf + kPData + kk * 256, 128, KV4 * 4),
-                           tc::sdesc(st + kStV + kk * 256, 128, KV4 * 4), id4_o,
-                           tmem + kColSFP + 8 * x + kk * 4, tmem + kColSFV + 8 * x + kk * 4,
-                           acc0 | (kk > 0));
+              tc::mma_nvf4_ta(dO, aP + kk * 8, tc::sdesc(st + kStV + kk * 256, 128, KV4 * 4), id4_o,
+                              tmem + kColSFP + 8 * x + kk * 4, tmem + kColSFV + 8 * x + kk * 4,
+                              acc0 | (kk > 0));
           }
           tc::mma_commit(&tb->p_free);
           tc::mma_commit(&bars->kv_empty[s]);
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t colO = x ? kColO1 : kColO0;
     TileBars* tb = &bars->tb[x];
-    uint8_t* pbuf = sm + kP0 + x * kPBytes;
+    const uint32_t colP = kColP + 32 * x;
     const int fpf = g.ny * g.nx;
     uint32_t gx = 0;                                     // blocks of this tile so far
     bool dead = false;                                   // a wait ran out: stop
@@ -570,10 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           jC = list_j(t + 65 + lane);
         }
         const int ecls = sm[kEdge + j];
-        if (t < n8)
-          softmax_block<D, BS, true>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
-        else
-          softmax_block<D, BS, false>(w, tb, sm, pbuf, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
+        softmax_block<D, BS>(t < n8, w, tb, sm, colP, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
       }
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
       if (!wait_bar(&tb->o_full, k & 1, w.err)) {
