@@ -61,9 +61,30 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-__device__ __forceinline__ float rcp_approx(float x) {
+// Pairs of fp32 values in one 64-bit register for the packed f32x2 instructions (two
+// lanes per instruction, each rounded as the scalar instruction would round it).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float lg2(float x) {
   float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -206,20 +227,23 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
     wait_bar(&tb->p_free, (gx - 1) & 1, w.err);
     tc::fence_after_sync();
   }
-  float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  // row-sum partials: keys 4i+0/4i+1 in sA, 4i+2/4i+3 in sB
+  f32x2 sA = pk2(0.0f, 0.0f), sB = pk2(0.0f, 0.0f);
+  const f32x2 c2 = pk2(c, c);
   if (FP8) {
+    const f32x2 b2 = pk2(bias, bias);
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
       uint32_t wd[4];
 #pragma unroll
       for (int e = 0; e < 16; e += 4) {
-        float p[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          p[u] = ex2(fmaf(s[16 * q + e + u], c, bias));
-          sum4[u] += p[u];
-        }
-        wd[e / 4] = (uint32_t)f32x2_to_e4m3x2(p[0], p[1]) | ((uint32_t)f32x2_to_e4m3x2(p[2], p[3]) << 16);
+        float x0, x1, x2, x3;
+        upk2(fma2(pk2(s[16 * q + e], s[16 * q + e + 1]), c2, b2), x0, x1);
+        upk2(fma2(pk2(s[16 * q + e + 2], s[16 * q + e + 3]), c2, b2), x2, x3);
+        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+        sA = add2(sA, pk2(p0, p1));
+        sB = add2(sB, pk2(p2, p3));
+        wd[e / 4] = (uint32_t)f32x2_to_e4m3x2(p0, p1) | ((uint32_t)f32x2_to_e4m3x2(p2, p3) << 16);
       }
       tc::tmem_st4(tmem + lane_base + colP + 4 * q, wd);
     }
@@ -227,25 +251,43 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
     uint32_t sfw[KV4 / 64];
 #pragma unroll
     for (int q = 0; q < KV4 / 64; ++q) sfw[q] = 0u;
-    // group scales first (independent chains): sigma = E4M3(448 p_max / 6), p_max from
-    // the group max
-    float rs[NG];
+    // Group scales first (independent chains): sigma = E4M3(448 p_max / 6), p_max from the
+    // group max. The E2M1 operand y = p448 / sigma is then taken as one exp2 with the
+    // group's shift -log2(sigma) folded into the bias, and the row sum gets sigma times
+    // the group's sum of y. A group with sigma = 0 keeps shift 0: its p448 are below a
+    // quarter, so their E2M1 codes are 0, and its sum is p448 itself.
+    float gb[NG], gs[NG];
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
       const uint32_t sc = f32_to_e4m3(ex2(fmaf(gm[q], c, bias)) * (1.0f / 6.0f));
       const float sg = e4m3_to_f32((uint8_t)sc);
-      rs[q] = sg > 0.0f ? rcp_approx(sg) : 0.0f;
+      gb[q] = sg > 0.0f ? bias - lg2(sg) : bias;
+      gs[q] = sg > 0.0f ? sg : 1.0f;
       sfw[q >> 2] |= sc << (8 * (q & 3));
     }
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
+      const f32x2 b2 = pk2(gb[q], gb[q]);
       float y[16];
+      f32x2 yA = pk2(0.0f, 0.0f), yB = pk2(0.0f, 0.0f);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float p = ex2(fmaf(s[16 * q + e], c, bias));
-        sum4[e & 3] += p;
-        y[e] = p * rs[q];
+      for (int e = 0; e < 16; e += 4) {
+        float x0, x1, x2, x3;
+        upk2(fma2(pk2(s[16 * q + e], s[16 * q + e + 1]), c2, b2), x0, x1);
+        upk2(fma2(pk2(s[16 * q + e + 2], s[16 * q + e + 3]), c2, b2), x2, x3);
+        y[e] = ex2(x0);
+        y[e + 1] = ex2(x1);
+        y[e + 2] = ex2(x2);
+        y[e + 3] = ex2(x3);
+        yA = add2(yA, pk2(y[e], y[e + 1]));
+        yB = add2(yB, pk2(y[e + 2], y[e + 3]));
       }
+      float a0, a1, b0, b1;
+      upk2(yA, a0, a1);
+      upk2(yB, b0, b1);
+      const float gsum = (a0 + a1) + (b0 + b1);
+      if (q & 1) sB = add2(sB, pk2(gs[q] * gsum, 0.0f));
+      else sA = add2(sA, pk2(gs[q] * gsum, 0.0f));
       tc::tmem_st2(tmem + lane_base + colP + 2 * q, f32x8_to_e2m1x8(y), f32x8_to_e2m1x8(y + 8));
     }
 #pragma unroll
@@ -258,7 +300,10 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
 #pragma unroll
     for (int q = 0; q < KV4 / 64; ++q) tc::tmem_st1(tmem + lane_base + sfp + 4 * q + (r >> 5), sfw[q]);
   }
-  l = fmaf(l, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+  float s0, s1, s2, s3;
+  upk2(sA, s0, s1);
+  upk2(sB, s2, s3);
+  l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
   // O row *= alpha (the previous P V of this tile has landed: waited above)
   if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) rescale_o<D>(tmem + lane_base + colO, alpha);
   m = m_new;
