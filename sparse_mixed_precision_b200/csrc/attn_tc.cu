@@ -77,6 +77,11 @@ __device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
   f32x2 d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -258,12 +263,19 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
     // quarter, so their E2M1 codes are 0, and its sum is p448 itself.
     float gb[NG], gs[NG];
 #pragma unroll
-    for (int q = 0; q < NG; ++q) {
-      const uint32_t sc = f32_to_e4m3(ex2(fmaf(gm[q], c, bias)) * (1.0f / 6.0f));
-      const float sg = e4m3_to_f32((uint8_t)sc);
-      gb[q] = sg > 0.0f ? bias - lg2(sg) : bias;
-      gs[q] = sg > 0.0f ? sg : 1.0f;
-      sfw[q >> 2] |= sc << (8 * (q & 3));
+    for (int q = 0; q < NG; q += 2) {                       // two groups at a time
+      float z0, z1;
+      upk2(fma2(pk2(gm[q], gm[q + 1]), pk2(c, c), pk2(bias, bias)), z0, z1);
+      upk2(mul2(pk2(ex2(z0), ex2(z1)), pk2(1.0f / 6.0f, 1.0f / 6.0f)), z0, z1);
+      const uint32_t sc2 = f32x2_to_e4m3x2(z0, z1);          // group q in the low byte
+      uint32_t h2;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)sc2));
+      const float2 sg = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+      gb[q] = sg.x > 0.0f ? bias - lg2(sg.x) : bias;
+      gb[q + 1] = sg.y > 0.0f ? bias - lg2(sg.y) : bias;
+      gs[q] = sg.x > 0.0f ? sg.x : 1.0f;
+      gs[q + 1] = sg.y > 0.0f ? sg.y : 1.0f;
+      sfw[q >> 2] |= sc2 << (8 * (q & 3));
     }
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
