@@ -44,10 +44,23 @@ __global__ void __launch_bounds__(256) k_vamax(const __nv_bfloat16* __restrict__
   float m[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = 0.0f;
-  const __nv_bfloat16* base = v + (size_t)bh * T * D;
-  for (int t = t0 + tr; t < t1; t += RSTEP) {
+  const __nv_bfloat16* base = v + (size_t)bh * T * D + cv * 8;
+  int t = t0 + tr;
+  for (; t + 3 * RSTEP < t1; t += 4 * RSTEP) {        // four loads in flight per thread
+    uint4 u[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) u[j] = ld_stream_u4(base + (size_t)(t + j * RSTEP) * D);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float f[8];
+      bf16x8_to_f32(u[j], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(f[i]));
+    }
+  }
+  for (; t < t1; t += RSTEP) {
     float f[8];
-    bf16x8_to_f32(ld_stream_u4(base + (size_t)t * D + cv * 8), f);
+    bf16x8_to_f32(ld_stream_u4(base + (size_t)t * D), f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(f[i]));
   }
@@ -59,6 +72,29 @@ __global__ void __launch_bounds__(256) k_vamax(const __nv_bfloat16* __restrict__
     for (int r = 0; r < RSTEP; ++r) a = fmaxf(a, red[r][c]);
     atomicMax(reinterpret_cast<unsigned int*>(vamax + (size_t)bh * D + c), __float_as_uint(a));
   }
+}
+
+// quant_fp4_group16 with the correctly rounded reciprocal of the group scale taken from a
+// table over the 128 non-negative E4M3 codes (filled with __frcp_rn of each code's value,
+// so the codes are the same bit for bit).
+__device__ __forceinline__ uint8_t quant_fp4_group16_tab(const float* y, uint32_t* packed2,
+                                                         const float* rcp_tab) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[i]));
+  const uint8_t sc = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+  if (sc != 0) {
+    const float r = rcp_tab[sc & 0x7F];
+    float z[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) z[i] = __fmul_rn(y[i], r);
+    packed2[0] = f32x8_to_e2m1x8(z);
+    packed2[1] = f32x8_to_e2m1x8(z + 8);
+  } else {
+    packed2[0] = 0u;
+    packed2[1] = 0u;
+  }
+  return sc;
 }
 
 // ---- K1: fused preparation of one (b, h, block) of Q, K (pool + quantise) or V ----
@@ -74,6 +110,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
   const int bs = g.bs;
   uint8_t* sfbuf = smem + (size_t)bs * RS * 2;             // up to 1 KB of group scales
   float* red = reinterpret_cast<float*>(sfbuf + 1024);      // reduction scratch / V scales
+  float* rcp_tab = red + 128;                               // 1/value of each E4M3 code
 
   const int n = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int tid = threadIdx.x;
@@ -107,6 +144,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
   }
   const int sfbytes = which < 2 ? (int)w.sf_qk : (int)w.sf_v;
   for (int i = tid; i < sfbytes / 4; i += 256) reinterpret_cast<uint32_t*>(sfbuf)[i] = 0u;
+  if (tid < 128) rcp_tab[tid] = tid > 0 ? __frcp_rn(e4m3_to_f32((uint8_t)tid)) : 0.0f;
   __syncthreads();
 
   if (which < 2) {
@@ -183,7 +221,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
                 ((uint32_t)f32x2_to_e4m3x2(y[4 * i + 2], y[4 * i + 3]) << 16);
       *reinterpret_cast<uint4*>(t8 + (size_t)u * 16) = make_uint4(p8[0], p8[1], p8[2], p8[3]);
       uint32_t p4[2];
-      const uint8_t sc = quant_fp4_group16(y, p4);
+      const uint8_t sc = quant_fp4_group16_tab(y, p4, rcp_tab);
       *reinterpret_cast<uint2*>(t4 + kmajor_off(r, kc * 8, D / 2)) = make_uint2(p4[0], p4[1]);
       sfbuf[sf_off(kc >> 2, r, kc & 3)] = sc;
     }
@@ -224,7 +262,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
         for (int i = 0; i < 16; ++i) y[i] = 0.0f;
       }
       uint32_t p4[2];
-      const uint8_t s4 = quant_fp4_group16(y, p4);
+      const uint8_t s4 = quant_fp4_group16_tab(y, p4, rcp_tab);
       *reinterpret_cast<uint2*>(t4 + kmajor_off(c, sc * 8, g.kv4 / 2)) = make_uint2(p4[0], p4[1]);
       sfbuf[sf_off(sc >> 2, c, sc & 3)] = s4;
     }
@@ -236,7 +274,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
 }
 
 size_t prepare_smem_bytes(const Geo& g) {
-  return (size_t)g.bs * (g.d + 8) * 2 + 1024 + 4 * 128;
+  return (size_t)g.bs * (g.d + 8) * 2 + 1024 + 4 * 128 + 4 * 128;
 }
 
 cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
