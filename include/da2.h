@@ -148,8 +148,16 @@ da2_status da2_forward(const da2_config* cfg, const void* q, const void* k, cons
 
 /* Host-buffer variant of da2_forward: copies q, k, v (host, bf16 [B,H,T,d]; pinned
    memory gives asynchronous copies) into the caller's device staging buffers dq, dk, dv,
-   runs the three stages and copies the result from dout back to out_host, all on
-   `stream`. Synchronises `stream` before returning so out_host is ready. */
+   runs the three stages and copies the result from dout back to out_host. Heads being
+   independent, it pipelines over up to 8 groups of heads: the copies in of one group and
+   the copy out of another overlap the stages of a third (three internal streams, two
+   sub-workspaces carved from ws, used alternately; each group's stages are exactly those
+   of da2_forward on a configuration of its heads, so out_host is bit-identical to
+   da2_forward's output). With fewer than 2 groups, or a workspace too small for two
+   sub-workspaces, it runs everything on `stream`. Work queued on `stream` before the call
+   runs first; the call synchronises `stream` before returning. Afterwards only the error
+   word of ws (da2_get_error with cfg) is meaningful; the rest of ws holds the groups'
+   layouts. ws_bytes must be at least da2_workspace_size(cfg). */
 da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const void* k_host,
                             const void* v_host, void* out_host, void* dq, void* dk,
                             void* dv, void* dout, void* ws, size_t ws_bytes,

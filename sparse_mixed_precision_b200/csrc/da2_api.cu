@@ -192,14 +192,12 @@ da2_status da2_forward(const da2_config* cfg, const void* q, const void* k, cons
   return da2_attention(cfg, ws, ws_bytes, out, stream);
 }
 
-da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const void* k_host,
-                            const void* v_host, void* out_host, void* dq, void* dk, void* dv,
-                            void* dout, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  const da2_status s0 = check_config(cfg);
-  if (s0 != DA2_OK) return s0;
-  if (!q_host || !k_host || !v_host || !out_host || !dq || !dk || !dv || !dout)
-    return DA2_ERR_INVALID_ARG;
-  const size_t bytes = (size_t)cfg->B * cfg->H * cfg->F * cfg->Hf * cfg->Wf * cfg->d * 2;
+namespace {
+
+// The whole path on one stream: copies in, three stages, copy out.
+da2_status forward_host_serial(const da2_config* cfg, const void* q_host, const void* k_host,
+                               const void* v_host, void* out_host, void* dq, void* dk, void* dv,
+                               void* dout, void* ws, size_t ws_bytes, cudaStream_t stream, size_t bytes) {
   cudaError_t e = cudaMemcpyAsync(dq, q_host, bytes, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, bytes, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, bytes, cudaMemcpyHostToDevice, stream);
@@ -209,6 +207,121 @@ da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const voi
   e = cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   return cuda_status(e);
+}
+
+constexpr int kHostGroups = 8;    // head groups the host-buffer path pipelines over
+
+}  // namespace
+
+// Heads are independent, so the host-buffer path runs as a pipeline over groups of heads:
+// the copies in of group g+1 and the copy out of group g-1 overlap the three stages of
+// group g (one stream each for copies in, compute and copies out; two sub-workspaces of
+// the caller's workspace used alternately). Every stage runs exactly as in da2_forward on
+// a configuration of that group's heads.
+da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const void* k_host,
+                            const void* v_host, void* out_host, void* dq, void* dk, void* dv,
+                            void* dout, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const da2_status s0 = check_config(cfg);
+  if (s0 != DA2_OK) return s0;
+  if (!q_host || !k_host || !v_host || !out_host || !dq || !dk || !dv || !dout)
+    return DA2_ERR_INVALID_ARG;
+  const size_t head_bytes = (size_t)cfg->F * cfg->Hf * cfg->Wf * cfg->d * 2;
+  const int BH = cfg->B * cfg->H;
+  const size_t bytes = head_bytes * BH;
+  size_t full_ws = 0;
+  if (da2_workspace_size(cfg, &full_ws) != DA2_OK || ws_bytes < full_ws) return DA2_ERR_WORKSPACE;
+
+  // group size: kHostGroups groups when there are enough heads and the two sub-workspaces
+  // (plus one error word per group) fit in the caller's workspace
+  const int hg = (BH + kHostGroups - 1) / kHostGroups;
+  const int G = (BH + hg - 1) / hg;
+  da2_config sub = *cfg;
+  sub.B = 1;
+  sub.H = hg;
+  size_t sub_ws = 0;
+  if (G < 2 || da2_workspace_size(&sub, &sub_ws) != DA2_OK)
+    return forward_host_serial(cfg, q_host, k_host, v_host, out_host, dq, dk, dv, dout, ws, ws_bytes, stream, bytes);
+  sub_ws = (sub_ws + 255) & ~size_t(255);
+  if (2 * sub_ws + 4 * (size_t)G > ws_bytes)
+    return forward_host_serial(cfg, q_host, k_host, v_host, out_host, dq, dk, dv, dout, ws, ws_bytes, stream, bytes);
+  uint8_t* ws8 = static_cast<uint8_t*>(ws);
+  uint32_t* err_acc = reinterpret_cast<uint32_t*>(ws8 + 2 * sub_ws);   // one word per group
+
+  cudaStream_t st_in = nullptr, st_cmp = nullptr, st_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in[kHostGroups] = {}, ev_cmp[kHostGroups] = {}, ev_end[3] = {};
+  da2_status status = DA2_OK;
+  cudaError_t e = cudaStreamCreateWithFlags(&st_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&st_cmp, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&st_out, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+  for (int g = 0; g < G && e == cudaSuccess; ++g) {
+    e = cudaEventCreateWithFlags(&ev_in[g], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_cmp[g], cudaEventDisableTiming);
+  }
+  for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&ev_end[i], cudaEventDisableTiming);
+  // everything queued on the caller's stream so far comes first
+  if (e == cudaSuccess) e = cudaEventRecord(ev_start, stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st_in, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st_cmp, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st_out, ev_start, 0);
+  for (int g = 0; g < G && e == cudaSuccess && status == DA2_OK; ++g) {
+    const int h0 = g * hg, nh = BH - h0 < hg ? BH - h0 : hg;
+    sub.H = nh;
+    const size_t off = head_bytes * h0, len = head_bytes * nh;
+    uint8_t* wsg = ws8 + (g & 1) * sub_ws;
+    e = cudaMemcpyAsync(static_cast<uint8_t*>(dq) + off, static_cast<const uint8_t*>(q_host) + off, len,
+                        cudaMemcpyHostToDevice, st_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<uint8_t*>(dk) + off, static_cast<const uint8_t*>(k_host) + off, len,
+                          cudaMemcpyHostToDevice, st_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<uint8_t*>(dv) + off, static_cast<const uint8_t*>(v_host) + off, len,
+                          cudaMemcpyHostToDevice, st_in);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in[g], st_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st_cmp, ev_in[g], 0);
+    if (e != cudaSuccess) break;
+    status = da2_forward(&sub, static_cast<uint8_t*>(dq) + off, static_cast<uint8_t*>(dk) + off,
+                         static_cast<uint8_t*>(dv) + off, static_cast<uint8_t*>(dout) + off, wsg, sub_ws, st_cmp);
+    if (status != DA2_OK) break;
+    // keep this group's error word before the sub-workspace is reused two groups later
+    da2_views vw;
+    da2_workspace_views(&sub, &vw);
+    e = cudaMemcpyAsync(err_acc + g, wsg + vw.err, 4, cudaMemcpyDeviceToDevice, st_cmp);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_cmp[g], st_cmp);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st_out, ev_cmp[g], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<uint8_t*>(out_host) + off, static_cast<const uint8_t*>(dout) + off, len,
+                          cudaMemcpyDeviceToHost, st_out);
+  }
+  // the caller's stream continues after all three
+  cudaError_t e2 = cudaSuccess;
+  cudaStream_t sts[3] = {st_in, st_cmp, st_out};
+  for (int i = 0; i < 3; ++i)
+    if (sts[i] && ev_end[i]) {
+      if (cudaEventRecord(ev_end[i], sts[i]) == cudaSuccess) cudaStreamWaitEvent(stream, ev_end[i], 0);
+    }
+  e2 = cudaStreamSynchronize(stream);
+  // fold the groups' error words into the error word of the workspace laid out for cfg
+  if (e == cudaSuccess && e2 == cudaSuccess && status == DA2_OK) {
+    uint32_t words[kHostGroups] = {};
+    e2 = cudaMemcpy(words, err_acc, 4 * (size_t)G, cudaMemcpyDeviceToHost);
+    uint32_t any = 0;
+    for (int g = 0; g < G; ++g) any |= words[g];
+    da2_views vfull;
+    da2_workspace_views(cfg, &vfull);
+    if (e2 == cudaSuccess) e2 = cudaMemcpy(ws8 + vfull.err, &any, 4, cudaMemcpyHostToDevice);
+  }
+  for (int g = 0; g < kHostGroups; ++g) {
+    if (ev_in[g]) cudaEventDestroy(ev_in[g]);
+    if (ev_cmp[g]) cudaEventDestroy(ev_cmp[g]);
+  }
+  for (int i = 0; i < 3; ++i)
+    if (ev_end[i]) cudaEventDestroy(ev_end[i]);
+  if (ev_start) cudaEventDestroy(ev_start);
+  for (int i = 0; i < 3; ++i)
+    if (sts[i]) cudaStreamDestroy(sts[i]);
+  if (status != DA2_OK) return status;
+  return cuda_status(e != cudaSuccess ? e : e2);
 }
 
 da2_status da2_get_error(void* ws, size_t ws_bytes, const da2_config* cfg, cudaStream_t stream,

@@ -211,3 +211,23 @@ def test_relative_error_against_dense_fp32_reported(capsys):
         rel = (got - ref).norm() / ref.norm()
         print(f"wan480 head {h}: rel-L2 vs dense fp32 attention = {rel.item():.4f}")
         assert rel < 0.5
+
+
+@pytest.mark.parametrize("name,heads", [("tiny", 0), ("wan720", 16)])
+def test_forward_host_pipeline_matches_forward(name, heads):
+    # da2_forward_host pipelines over groups of heads (copies overlapping compute); its
+    # host output must equal da2_forward's device output bit for bit
+    w = WORKLOADS[name] if heads == 0 else scaled(WORKLOADS[name], H=heads)
+    q, k, v = generate(w, device="cuda")
+    cfg = da2.config(w)
+    ws = torch.empty(da2.workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    da2.forward(cfg, q, k, v, out, ws)
+    torch.cuda.synchronize()
+    assert da2.get_error(cfg, ws) == 0
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    oh = torch.full(q.shape, float("nan"), dtype=q.dtype).pin_memory()
+    dq, dk, dv, dout = (torch.empty_like(q) for _ in range(4))
+    da2.forward_host(cfg, qh, kh, vh, oh, dq, dk, dv, dout, ws)
+    assert da2.get_error(cfg, ws) == 0
+    assert torch.equal(oh, out.cpu())
