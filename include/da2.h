@@ -68,7 +68,12 @@ enum {
   DA2_FLAG_EXPORT_SCORES = 1,
   /* Drop the ln(valid tokens) term of the draft logits (the maps then rank by average
      token affinity instead of block mass). */
-  DA2_FLAG_NO_MASS_CORRECTION = 2
+  DA2_FLAG_NO_MASS_CORRECTION = 2,
+  /* q, k, v and out are token-major, bf16 [B,T,H,d] (the heads of one token adjacent, as
+     a fused QKV projection usually leaves them) instead of [B,H,T,d]; read and written in
+     place, results identical. da2_forward_host then runs unpipelined. (The pages fix no
+     tensor layout.) */
+  DA2_FLAG_LAYOUT_BTHD = 4
 };
 
 typedef enum da2_status {
@@ -125,7 +130,8 @@ da2_status da2_workspace_size(const da2_config* cfg, size_t* bytes);
 /* Geometry and region offsets for `cfg` (host only, no CUDA call). */
 da2_status da2_workspace_views(const da2_config* cfg, da2_views* views);
 
-/* Operand preparation. q, k, v: device bf16 [B,H,T,d]; ws: device workspace of at least
+/* Operand preparation. q, k, v: device bf16 [B,H,T,d] ([B,T,H,d] with
+   DA2_FLAG_LAYOUT_BTHD); ws: device workspace of at least
    da2_workspace_size bytes. Writes every operand, scale and pooled region of ws and
    clears its error word. Asynchronous on `stream`. */
 da2_status da2_prepare(const da2_config* cfg, const void* q, const void* k, const void* v,
@@ -137,7 +143,7 @@ da2_status da2_draft_select(const da2_config* cfg, void* ws, size_t ws_bytes,
                             cudaStream_t stream);
 
 /* Mixed-precision block-sparse attention on a prepared and selected workspace. out:
-   device bf16 [B,H,T,d] (every element is written). Bounded device waits that run out
+   device bf16 [B,H,T,d] ([B,T,H,d] with DA2_FLAG_LAYOUT_BTHD; every element is written). Bounded device waits that run out
    set the workspace error word (read it with da2_get_error). Asynchronous. */
 da2_status da2_attention(const da2_config* cfg, void* ws, size_t ws_bytes, void* out,
                          cudaStream_t stream);
@@ -149,7 +155,7 @@ da2_status da2_forward(const da2_config* cfg, const void* q, const void* k, cons
 /* Host-buffer variant of da2_forward: copies q, k, v (host, bf16 [B,H,T,d]; pinned
    memory gives asynchronous copies) into the caller's device staging buffers dq, dk, dv,
    runs the three stages and copies the result from dout back to out_host. Heads being
-   independent, it pipelines over up to 8 groups of heads: the copies in of one group and
+   independent, it pipelines over up to 16 groups of heads: the copies in of one group and
    the copy out of another overlap the stages of a third (three internal streams, two
    sub-workspaces carved from ws, used alternately; each group's stages are exactly those
    of da2_forward on a configuration of its heads, so out_host is bit-identical to

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libda2.so")
 
 FLAG_EXPORT_SCORES = 1
 FLAG_NO_MASS_CORRECTION = 2
+FLAG_LAYOUT_BTHD = 4          # q, k, v, out token-major [B, T, H, d]
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned pointer",
           4: "workspace too small", 5: "CUDA error", 6: "device error word set",

@@ -592,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       if (row_ok) {
         const int f = i / fpf, rem = i - f * fpf, by = rem / g.nx, bx = rem - by * g.nx;
         const size_t tk = (size_t)f * g.Hf * g.Wf + (size_t)(by * g.ph + wy) * g.Wf + bx * g.pw + wx;
-        orow = out + ((size_t)bh * g.T + tk) * D;
+        orow = out + tok_off(g, bh, tk);
       }
       if (nb == 0) {
         if (row_ok)

@@ -17,7 +17,19 @@ struct Geo {
   int ny, nx, N, bs, T, Tp, n8, n4, kv4;
   float sm_scale;
   int flags;
+  int bthd;   // q, k, v, out token-major [B,T,H,d] instead of [B,H,T,d]
 };
+
+// Element offset of token t, channel 0 of head bh = b*H + h in a q/k/v/out tensor.
+__host__ __device__ __forceinline__ size_t tok_off(const Geo& g, int bh, size_t t) {
+  if (!g.bthd) return ((size_t)bh * g.T + t) * g.d;
+  const int b = bh / g.H, h = bh - b * g.H;
+  return (((size_t)b * g.T + t) * g.H + h) * g.d;
+}
+// Elements between consecutive tokens of one head.
+__host__ __device__ __forceinline__ size_t tok_stride(const Geo& g) {
+  return g.bthd ? (size_t)g.H * g.d : (size_t)g.d;
+}
 
 // Workspace base pointers, resolved on the host.
 struct Ws {

@@ -27,6 +27,8 @@ da2_status check_config(const da2_config* c) {
     return DA2_ERR_INVALID_ARG;
   if (c->pct_fp8 < 0 || c->pct_fp4 < 0 || c->pct_fp8 + c->pct_fp4 > 100) return DA2_ERR_INVALID_ARG;
   if (!(c->sm_scale >= 0.0f) || std::isinf(c->sm_scale)) return DA2_ERR_INVALID_ARG;
+  if (c->flags & ~(DA2_FLAG_EXPORT_SCORES | DA2_FLAG_NO_MASS_CORRECTION | DA2_FLAG_LAYOUT_BTHD))
+    return DA2_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return DA2_ERR_UNSUPPORTED;
   const long bs = (long)c->ph * c->pw;
   if (bs != 32 && bs != 64 && bs != 128) return DA2_ERR_UNSUPPORTED;
@@ -90,6 +92,7 @@ Geo make_geo(const da2_config* c, const da2_views& v) {
   g.T = v.T; g.Tp = v.Tp; g.n8 = v.n8; g.n4 = v.n4; g.kv4 = v.kv4;
   g.sm_scale = c->sm_scale > 0.0f ? c->sm_scale : 1.0f / std::sqrt((float)c->d);
   g.flags = c->flags;
+  g.bthd = (c->flags & DA2_FLAG_LAYOUT_BTHD) ? 1 : 0;
   return g;
 }
 
@@ -209,7 +212,7 @@ da2_status forward_host_serial(const da2_config* cfg, const void* q_host, const 
   return cuda_status(e);
 }
 
-constexpr int kHostGroups = 8;    // head groups the host-buffer path pipelines over
+constexpr int kHostGroups = 16;   // head groups the host-buffer path pipelines over
 
 }  // namespace
 
@@ -239,7 +242,7 @@ da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const voi
   sub.B = 1;
   sub.H = hg;
   size_t sub_ws = 0;
-  if (G < 2 || da2_workspace_size(&sub, &sub_ws) != DA2_OK)
+  if (G < 2 || (cfg->flags & DA2_FLAG_LAYOUT_BTHD) || da2_workspace_size(&sub, &sub_ws) != DA2_OK)
     return forward_host_serial(cfg, q_host, k_host, v_host, out_host, dq, dk, dv, dout, ws, ws_bytes, stream, bytes);
   sub_ws = (sub_ws + 255) & ~size_t(255);
   if (2 * sub_ws + 4 * (size_t)G > ws_bytes)

@@ -32,9 +32,11 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 u, float* f) {
 
 // ---- K0: amax of V over all tokens, per (b, h, channel) ----
 // grid (chunks, B*H); vamax must be zero on entry (non-negative floats compare as uints).
-template <int D>
-__global__ void __launch_bounds__(256) k_vamax(const __nv_bfloat16* __restrict__ v,
-                                               float* __restrict__ vamax, int T, int chunk) {
+// BTHD: q, k, v token-major [B,T,H,d] (token stride H*D) instead of [B,H,T,d] (stride D).
+template <int D, bool BTHD>
+__global__ void __launch_bounds__(256) k_vamax(Geo g, const __nv_bfloat16* __restrict__ v,
+                                               float* __restrict__ vamax, int chunk) {
+  const int T = g.T;
   constexpr int VPR = D / 8;          // 16-byte vectors per token
   constexpr int RSTEP = 256 / VPR;    // tokens per sweep
   __shared__ float red[RSTEP][D + 1];
@@ -44,12 +46,13 @@ __global__ void __launch_bounds__(256) k_vamax(const __nv_bfloat16* __restrict__
   float m[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = 0.0f;
-  const __nv_bfloat16* base = v + (size_t)bh * T * D + cv * 8;
+  const __nv_bfloat16* base = v + tok_off(g, bh, 0) + cv * 8;
+  const size_t ts = BTHD ? (size_t)g.H * D : (size_t)D;
   int t = t0 + tr;
   for (; t + 3 * RSTEP < t1; t += 4 * RSTEP) {        // four loads in flight per thread
     uint4 u[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) u[j] = ld_stream_u4(base + (size_t)(t + j * RSTEP) * D);
+    for (int j = 0; j < 4; ++j) u[j] = ld_stream_u4(base + (size_t)(t + j * RSTEP) * ts);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float f[8];
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(256) k_vamax(const __nv_bfloat16* __restrict__
   }
   for (; t < t1; t += RSTEP) {
     float f[8];
-    bf16x8_to_f32(ld_stream_u4(base + (size_t)t * D), f);
+    bf16x8_to_f32(ld_stream_u4(base + (size_t)t * ts), f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(f[i]));
   }
@@ -99,7 +102,7 @@ __device__ __forceinline__ uint8_t quant_fp4_group16_tab(const float* y, uint32_
 
 // ---- K1: fused preparation of one (b, h, block) of Q, K (pool + quantise) or V ----
 // grid (N, B*H, 3); blockIdx.z: 0 = Q, 1 = K, 2 = V.
-template <int D>
+template <int D, bool BTHD>
 __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat16* __restrict__ q,
                                                  const __nv_bfloat16* __restrict__ k,
                                                  const __nv_bfloat16* __restrict__ v) {
@@ -121,7 +124,8 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
   const int hv = min(g.ph, g.Hf - y0), wv = min(g.pw, g.Wf - x0);
 
   // stage the window (padded slots zero)
-  const __nv_bfloat16* sbase = src + (size_t)bh * g.T * D;
+  const __nv_bfloat16* sbase = src + tok_off(g, bh, 0);
+  const size_t ts = BTHD ? (size_t)g.H * D : (size_t)D;
   {
     // slot s = wy*pw + wx advances by a fixed step per iteration: step the window
     // coordinates instead of dividing every time
@@ -134,7 +138,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
       uint4 val = make_uint4(0u, 0u, 0u, 0u);
       if (wy < hv && wx < wv) {
         const size_t t = (size_t)f * g.Hf * g.Wf + (size_t)(y0 + wy) * g.Wf + (x0 + wx);
-        val = ld_stream_u4(sbase + t * D + cv * 8);
+        val = ld_stream_u4(sbase + t * ts + cv * 8);
       }
       *reinterpret_cast<uint4*>(X + sl * RS + cv * 8) = val;
       wx += dx;
@@ -291,12 +295,18 @@ cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void*
   const auto* qb = static_cast<const __nv_bfloat16*>(q);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
   const auto* vb = static_cast<const __nv_bfloat16*>(v);
-  if (g.d == 128) {
-    k_vamax<128><<<g0, 256, 0, st>>>(vb, w.vamax, g.T, chunk);
-    k_prepare<128><<<g1, 256, smem, st>>>(g, w, qb, kb, vb);
+  if (g.d == 128 && !g.bthd) {
+    k_vamax<128, false><<<g0, 256, 0, st>>>(g, vb, w.vamax, chunk);
+    k_prepare<128, false><<<g1, 256, smem, st>>>(g, w, qb, kb, vb);
+  } else if (g.d == 128) {
+    k_vamax<128, true><<<g0, 256, 0, st>>>(g, vb, w.vamax, chunk);
+    k_prepare<128, true><<<g1, 256, smem, st>>>(g, w, qb, kb, vb);
+  } else if (!g.bthd) {
+    k_vamax<64, false><<<g0, 256, 0, st>>>(g, vb, w.vamax, chunk);
+    k_prepare<64, false><<<g1, 256, smem, st>>>(g, w, qb, kb, vb);
   } else {
-    k_vamax<64><<<g0, 256, 0, st>>>(vb, w.vamax, g.T, chunk);
-    k_prepare<64><<<g1, 256, smem, st>>>(g, w, qb, kb, vb);
+    k_vamax<64, true><<<g0, 256, 0, st>>>(g, vb, w.vamax, chunk);
+    k_prepare<64, true><<<g1, 256, smem, st>>>(g, w, qb, kb, vb);
   }
   return cudaGetLastError();
 }

@@ -61,6 +61,15 @@ def test_invalid_configs_rejected(change, status):
     assert da2.lib().da2_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == status
 
 
+def test_flags_checked_and_layout_flag_keeps_the_workspace():
+    L = da2.lib()
+    n = ctypes.c_size_t()
+    w = WORKLOADS["tiny"]
+    assert L.da2_workspace_size(ctypes.byref(da2.config(w, flags=8)), ctypes.byref(n)) == 1
+    # the token-major layout changes where q/k/v/out live, not the workspace
+    assert da2.workspace_views(da2.config(w, flags=da2.FLAG_LAYOUT_BTHD)) == da2.workspace_views(da2.config(w))
+
+
 def test_stage_calls_reject_bad_pointers_without_touching_the_device():
     L = da2.lib()
     cfg = da2.config(WORKLOADS["tiny"])

@@ -231,3 +231,30 @@ def test_forward_host_pipeline_matches_forward(name, heads):
     da2.forward_host(cfg, qh, kh, vh, oh, dq, dk, dv, dout, ws)
     assert da2.get_error(cfg, ws) == 0
     assert torch.equal(oh, out.cpu())
+
+
+@pytest.mark.parametrize("name,heads", [("tiny", 0), ("wan480", 4)])
+def test_token_major_layout_matches(name, heads):
+    # DA2_FLAG_LAYOUT_BTHD reads q, k, v and writes out as [B, T, H, d] in place: the
+    # prepared workspace must be byte-identical and the output the same values
+    w = WORKLOADS[name] if heads == 0 else scaled(WORKLOADS[name], H=heads)
+    q, k, v = generate(w, device="cuda")
+    cfg = da2.config(w)
+    ws = torch.zeros(da2.workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    da2.forward(cfg, q, k, v, out, ws)
+    cfg_t = da2.config(w, flags=da2.FLAG_LAYOUT_BTHD)
+    ws_t = torch.zeros_like(ws)
+    qt, kt, vt = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+    out_t = torch.full_like(qt, float("nan"))
+    da2.forward(cfg_t, qt, kt, vt, out_t, ws_t)
+    torch.cuda.synchronize()
+    assert da2.get_error(cfg, ws) == 0 and da2.get_error(cfg_t, ws_t) == 0
+    assert torch.equal(ws, ws_t)
+    assert torch.equal(out_t.transpose(1, 2), out)
+    # the host-buffer path takes the same layout (unpipelined)
+    oh = torch.empty(qt.shape, dtype=qt.dtype).pin_memory()
+    dq, dk, dv, dout = (torch.empty_like(qt) for _ in range(4))
+    da2.forward_host(cfg_t, qt.cpu().pin_memory(), kt.cpu().pin_memory(), vt.cpu().pin_memory(), oh,
+                     dq, dk, dv, dout, ws_t)
+    assert torch.equal(oh, out_t.cpu())
