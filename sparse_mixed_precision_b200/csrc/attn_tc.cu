@@ -14,8 +14,10 @@
 //   m_new = max(m, rowmax(S * s_q s_k sm_scale)), padded keys masked
 //   l = l 2^(m-m_new) + sum p,  p = 2^(S' - m_new)  (log2 domain)
 //   O = O 2^(m-m_new)        (only when the max moved, done in TMEM by the softmax warps)
-//   P~ = E4M3(448 p) or E2M1(448 p / sigma) with sigma = E4M3(amax16 / 6) per 16 keys
-//   O += P~ V_j'             same MMA kind as the block, accumulating into the one O.
+//   P~ = E4M3(448 p) or E2M1(448 p / sigma) with sigma = E4M3(amax16 / 6) per 16 keys,
+//                            written to tensor memory by the softmax threads
+//   O += P~ V_j'             same MMA kind as the block (A = P~ read from tensor memory),
+//                            accumulating into the one O.
 // Epilogue: out = O s_v / (448 l) in bf16, written to the tokens' original positions.
 //
 // Two query tiles (work items) per CTA, processed as a ping-pong: while one tile's
@@ -29,14 +31,15 @@
 //   warp 9      producer: 1-D bulk copies of the pre-tiled Q/K/V operand tiles and scales
 //   warp 10     MMA issue for tile B (one thread)
 //   warp 11     idle
-// Tensor memory: O of each tile, ONE S region the two tiles take in turns, and scale
-// factors. Each tile's issuer runs S(0), then per block t: S(t+1), PV(t); the S region is
+// Tensor memory: O of each tile, ONE S region the two tiles take in turns, scale factors
+// and each tile's P~. Each tile's issuer runs S(0), then per block t: S(t+1), PV(t); the S region is
 // taken in the order S_A(t), S_B(t), S_A(t+1), ..., each S waiting until the softmax of
 // the previous owner has read its own. K/V stages are filled in that S order and released
 // after their P V.
-// Every mbarrier wait is bounded; a wait that runs out sets the workspace error word, each
-// role stops issuing work, the producer waits for its copies in flight and the MMA thread
-// for its MMAs, and the kernel frees its tensor memory and exits.
+// Every mbarrier wait is bounded; a wait that runs out sets the workspace error word; the
+// producer and the issuers stop issuing work, the producer waits for its copies in flight
+// and the issuers for their MMAs, the softmax warps run through the rest of their round
+// without waiting, and the kernel frees its tensor memory and exits.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -177,12 +180,13 @@ __device__ __noinline__ void rescale_o(uint32_t taddr, float alpha) {
   tc::tmem_wait_st();
 }
 
-// One KV block of one query row of a tile (softmax warps). The S row is read once from
-// the shared S region (which is released at once) -> group maxima -> row max -> alpha ->
-// one fused loop computing p448 = 2^(S c + log2 448 - m_new), the row sum and the
-// quantised P bytes (E4M3, or E2M1 with an E4M3 scale per 16 keys) stored straight into
-// the tile's P buffer -> O rescale by alpha in TMEM when the max moved (after the tile's
-// previous P V has landed) -> P ready.
+// One KV block of one query row of a tile (softmax warps; FP8 selects the block's
+// precision). The S row is read once from the shared S region (which is released at once)
+// -> group maxima -> row max -> alpha -> one fused loop computing p448 = 2^(S c + log2 448
+// - m_new), the row sum and the quantised P (E4M3, or E2M1 with an E4M3 scale per 16
+// keys), stored with tcgen05.st into the tile's P columns of tensor memory (after the
+// tile's previous P V has landed) -> O rescale by alpha in TMEM when the max moved -> P
+// ready.
 // gx counts this tile's blocks over the whole launch. A wait that runs out does not stop
 // the block (checking here costs the loop several percent): after a timeout every later
 // wait returns at once, so the rest of the round runs through without waiting and the
@@ -227,7 +231,7 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
   const float m_new = fmaxf(m, mh * c);
   const float alpha = ex2(m - m_new);
   const float bias = kLog2_448 - m_new;
-  // the P buffer (and O) are free once this tile's previous P V has completed
+  // the tile's P columns (and O) are free once its previous P V has completed
   if (t > 0) {
     wait_bar(&tb->p_free, (gx - 1) & 1, w.err);
     tc::fence_after_sync();
