@@ -258,3 +258,26 @@ def test_token_major_layout_matches(name, heads):
     da2.forward_host(cfg_t, qt.cpu().pin_memory(), kt.cpu().pin_memory(), vt.cpu().pin_memory(), oh,
                      dq, dk, dv, dout, ws_t)
     assert torch.equal(oh, out_t.cpu())
+
+
+@pytest.mark.parametrize("kw", [
+    dict(d=128),                                    # d 128, 32-token blocks
+    dict(ph=8, pw=8, Hf=16, Wf=32),                 # d 64, 64-token blocks
+    dict(ph=8, pw=16, Hf=16, Wf=32),                # d 64, 128-token blocks
+    dict(F=2, Hf=13, Wf=29),                        # short windows in both directions
+    dict(d=128, ph=8, pw=16, F=2, Hf=21, Wf=37, sinks=2),      # 128-token blocks, both edges
+], ids=["d128-bs32", "d64-bs64", "d64-bs128", "edges-bs32", "edges-d128-bs128"])
+def test_small_shapes_full_parity(kw):
+    # every instantiation of the kernels and both kinds of edge window, checked in full
+    w = scaled(WORKLOADS["tiny"], name="tiny-" + "-".join(f"{k}{v}" for k, v in kw.items()), **kw)
+    q, k, v = generate(w, device="cuda")
+    cfg, views, ws, out = run_cuda(w, q, k, v)
+    rd = WsReader(ws, views, w.d)
+    g = O.geometry(scaled(w, B=1, H=1))
+    for h in range(w.H):
+        qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+        P = check_prep(w, views, rd, h, qh, kh, vh)
+        l8, l4, _ = check_selection(views, rd, h, P, g)
+        check_attention(w, views, P, l8[0], l4[0], out[0, h].float().cpu().numpy(),
+                        list(range(g.N)), g)
+    assert torch.isfinite(out).all()
