@@ -94,29 +94,6 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t code) {
   return (code & 8u) ? -mag : mag;
 }
 
-// Quantise one group of 16 values y (already divided by their outer scale) to E2M1 with an
-// E4M3 group scale: sigma = E4M3(amax16 / 6); codes = E2M1(y * (1/sigma)); a group whose
-// sigma is zero is all zero codes. Writes 8 bytes of packed codes and returns sigma's byte.
-__device__ __forceinline__ uint8_t quant_fp4_group16(const float* y, uint32_t* packed2) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[i]));
-  const uint8_t sc = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
-  const float sig = e4m3_to_f32(sc);
-  if (sig > 0.0f) {
-    const float r = __frcp_rn(sig);
-    float z[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) z[i] = __fmul_rn(y[i], r);
-    packed2[0] = f32x8_to_e2m1x8(z);
-    packed2[1] = f32x8_to_e2m1x8(z + 8);
-  } else {
-    packed2[0] = 0u;
-    packed2[1] = 0u;
-  }
-  return sc;
-}
-
 __device__ __forceinline__ void set_error(uint32_t* err, uint32_t bits) {
   if (err) atomicOr(err, bits);
 }

@@ -77,9 +77,11 @@ __global__ void __launch_bounds__(256) k_vamax(Geo g, const __nv_bfloat16* __res
   }
 }
 
-// quant_fp4_group16 with the correctly rounded reciprocal of the group scale taken from a
-// table over the 128 non-negative E4M3 codes (filled with __frcp_rn of each code's value,
-// so the codes are the same bit for bit).
+// Quantise one group of 16 values y (already divided by their outer scale) to E2M1 with an
+// E4M3 group scale: sigma = E4M3(amax16 / 6); codes = E2M1(y * (1/sigma)), the correctly
+// rounded reciprocal taken from a table over the 128 non-negative E4M3 codes (filled with
+// __frcp_rn of each code's value); a group whose sigma is zero is all zero codes. Writes 8
+// bytes of packed codes and returns sigma's byte.
 __device__ __forceinline__ uint8_t quant_fp4_group16_tab(const float* y, uint32_t* packed2,
                                                          const float* rcp_tab) {
   float amax = 0.0f;
