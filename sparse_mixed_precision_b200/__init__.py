@@ -8,6 +8,12 @@ come from PyTorch); the library itself allocates nothing.
     ws  = torch.empty(workspace_size(cfg), dtype=torch.uint8, device="cuda")
     prepare(cfg, q, k, v, ws); draft_select(cfg, ws); attention(cfg, ws, out)
 
+Token-major activations ([B, T, H, d], heads of one token adjacent) go in as they are with
+`config(w, flags=FLAG_LAYOUT_BTHD)`. Sequence-parallel callers (each rank holding T/P of
+the tokens) exchange to all tokens of H/P heads with `seqpar.seq_to_heads` before the call
+and back with `seqpar.heads_to_seq` after it. `forward_host` takes pinned host buffers and
+overlaps the copies with the compute over groups of heads.
+
 The extension must be built first (`python -m sparse_mixed_precision_b200.build` or
 `__graft_entry__.build()`); there is no fallback when it is missing.
 """
