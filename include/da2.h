@@ -33,7 +33,9 @@
  *  - Budgets: n8 = floor((pct_fp8*N + 50)/100) FP8 KV blocks and n4 = floor(((pct_fp8 +
  *    pct_fp4)*N + 50)/100) - n8 FP4 KV blocks per query block; the rest are skipped.
  *  - Memory ownership: the caller allocates q, k, v, out and the workspace (device memory,
- *    size from da2_workspace_size); the library allocates nothing and keeps no state.
+ *    size from da2_workspace_size); the library allocates no device memory and keeps no
+ *    state (da2_forward_host creates and destroys three streams and a few events per call;
+ *    da2_forward_noalloc uses a static device array of the library image).
  *  - Every call is asynchronous on `stream` (0 = legacy default stream) except the ones
  *    documented as synchronising. Argument errors are returned before anything is
  *    enqueued; a failed launch returns DA2_ERR_CUDA (see cudaGetLastError for detail).

@@ -2,7 +2,7 @@
 
 Argument marshalling only: every step of the path runs in the CUDA library. The names
 follow the C ABI in include/da2.h. Tensors are torch tensors (device memory and streams
-come from PyTorch); the library itself allocates nothing.
+come from PyTorch); the library itself allocates no device memory.
 
     cfg = config(workload)                      # da2_config from a synth.Workload
     ws  = torch.empty(workspace_size(cfg), dtype=torch.uint8, device="cuda")
