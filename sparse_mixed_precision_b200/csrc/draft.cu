@@ -67,22 +67,24 @@ __device__ void warp_radix_select(const uint32_t* keys, int n, int kth, uint32_t
   need = remaining;
 }
 
+constexpr int kDraftThreads = 512, kDraftWarps = kDraftThreads / 32;
+
 template <int D>
-__global__ void __launch_bounds__(256) k_draft_select(Geo g, Ws w, int R) {
+__global__ void __launch_bounds__(kDraftThreads) k_draft_select(Geo g, Ws w, int R) {
   extern __shared__ __align__(16) float dsm[];
   const int N = g.N;
   float* qa = dsm;                 // [R][D]
   float* qm = qa + R * D;          // [R][D]
   float* la = qm + R * D;          // [R][N]  avg logits, later the score
   float* lm = la + R * N;          // [R][N]  max logits
-  uint32_t* hist = reinterpret_cast<uint32_t*>(lm + R * N);  // [8][256]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(lm + R * N);  // [warps][256]
   const int bh = blockIdx.y, i0 = blockIdx.x * R;
   const int rows = min(R, N - i0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   const float* qavg = w.qavg + ((size_t)bh * N + i0) * D;
   const float* qmax = w.qmax + ((size_t)bh * N + i0) * D;
-  for (int u = tid; u < R * D / 4; u += 256) {
+  for (int u = tid; u < R * D / 4; u += kDraftThreads) {
     const bool ok = u < rows * D / 4;
     reinterpret_cast<float4*>(qa)[u] = ok ? reinterpret_cast<const float4*>(qavg)[u] : make_float4(0, 0, 0, 0);
     reinterpret_cast<float4*>(qm)[u] = ok ? reinterpret_cast<const float4*>(qmax)[u] : make_float4(0, 0, 0, 0);
@@ -93,7 +95,7 @@ __global__ void __launch_bounds__(256) k_draft_select(Geo g, Ws w, int R) {
   const int fpf = g.ny * g.nx;
   const float* kavg = w.kavg + (size_t)bh * N * D;
   const float* kmax = w.kmax + (size_t)bh * N * D;
-  for (int j = tid; j < N; j += 256) {
+  for (int j = tid; j < N; j += kDraftThreads) {
     float aa[16], am[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) { aa[r] = 0.0f; am[r] = 0.0f; }
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(256) k_draft_select(Geo g, Ws w, int R) {
 
   const int nk = g.n8 + g.n4;
   uint32_t* h = hist + warp * 256;
-  for (int r = warp; r < rows; r += 8) {
+  for (int r = warp; r < rows; r += kDraftWarps) {
     float* ra = la + r * N;
     float* rm = lm + r * N;
     // two row softmaxes, averaged
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(256) k_draft_select(Geo g, Ws w, int R) {
 }
 
 size_t draft_smem_bytes(const Geo& g, int R) {
-  return (size_t)(2 * R * g.d + 2 * R * g.N) * 4 + 8 * 256 * 4;
+  return (size_t)(2 * R * g.d + 2 * R * g.N) * 4 + kDraftWarps * 256 * 4;
 }
 
 int draft_rows_per_cta(const Geo& g) {
@@ -213,11 +215,11 @@ cudaError_t launch_draft_select(const Geo& g, const Ws& w, cudaStream_t st) {
   if (g.d == 128) {
     e = cudaFuncSetAttribute(k_draft_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_draft_select<128><<<grid, 256, smem, st>>>(g, w, R);
+    k_draft_select<128><<<grid, kDraftThreads, smem, st>>>(g, w, R);
   } else {
     e = cudaFuncSetAttribute(k_draft_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_draft_select<64><<<grid, 256, smem, st>>>(g, w, R);
+    k_draft_select<64><<<grid, kDraftThreads, smem, st>>>(g, w, R);
   }
   return cudaGetLastError();
 }
