@@ -61,6 +61,25 @@ def test_invalid_configs_rejected(change, status):
     assert da2.lib().da2_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == status
 
 
+def test_config_limits_and_degenerate_budgets():
+    L = da2.lib()
+    n = ctypes.c_size_t()
+    w = WORKLOADS["tiny"]
+    def status(cfg):
+        return L.da2_workspace_size(ctypes.byref(cfg), ctypes.byref(n))
+    # 4096 blocks is the largest supported per (b, h); one more is refused
+    assert status(da2.config(scaled(w, F=32, Hf=64, Wf=64, ph=4, pw=8))) == 0      # N = 4096
+    assert status(da2.config(scaled(w, F=33, Hf=64, Wf=64, ph=4, pw=8))) == 2      # N = 4224
+    # a negative or non-finite softmax scale is an argument error; 0 selects 1/sqrt(d)
+    assert status(da2.config(w, sm_scale=-1.0)) == 1
+    assert status(da2.config(w, sm_scale=float("inf"))) == 1
+    assert status(da2.config(w, sm_scale=0.0)) == 0
+    # budgets: nothing kept, everything FP8, everything FP4 are all valid
+    for f8, f4 in ((0, 0), (100, 0), (0, 100)):
+        v = da2.workspace_views(da2.config(scaled(w, pct_fp8=f8, pct_fp4=f4)))
+        assert v["n8"] == v["N"] * f8 // 100 and v["n4"] == v["N"] * f4 // 100
+
+
 def test_flags_checked_and_layout_flag_keeps_the_workspace():
     L = da2.lib()
     n = ctypes.c_size_t()
