@@ -49,6 +49,18 @@ def executed_flops(w):
     return rows * n8 * per, rows * (nk - n8) * per
 
 
+def draft_flops(w) -> float:
+    """Algorithmic FLOP of the draft maps: two (N x d) @ (d x N) logit products per head."""
+    import math as _m
+    N = w.F * _m.ceil(w.Hf / w.ph) * _m.ceil(w.Wf / w.pw)
+    return 2.0 * 2.0 * N * N * w.d * w.B * w.H
+
+
+def fp32_fma_peak_tflops(sm_mhz: float, sms: int = 148) -> float:
+    """fp32 FMA peak from the unit counts: 128 FMA lanes per SM per clock, 2 FLOP each."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def prep_bytes(w) -> float:
     """Algorithmic HBM bytes of the preparation stage (reads once, writes once)."""
     import math as _m
@@ -88,6 +100,15 @@ def attention_traffic(w):
     if rec.get("source_sha256") != attn_source_hash() or rec.get("workload") != w.name:
         return None
     return rec["attention_dram_bytes"] * (w.B * w.H) / rec["captured_bh"]
+
+
+def draft_alu_entry(w, draft_ms: float, peaks: dict) -> dict:
+    """The draft stage against its own bound: fp32 FMA throughput (ALU-bound; it reads only
+    the 52 MB of pooled vectors), peak from the unit counts at the measured max SM clock."""
+    peak = fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
+    achieved = draft_flops(w) / (draft_ms * 1e-3) / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "note": "fp32 FMA peak = 148 SMs x 128 lanes x 2 FLOP x SM clock"}
 
 
 def load_peaks():
@@ -381,6 +402,7 @@ def main():
                              f" at {p8:.0f} / {p4:.0f} TFLOP/s = 2x / 4x {src} sustained bf16)"},
         "prepare_hbm": {"achieved_gbs": pb / (prep_ms * 1e-3) / 1e9, "peak_gbs": peaks["hbm_gbs"],
                         "frac": pb / (prep_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "draft_alu": draft_alu_entry(w, statistics.mean(stage["draft_select"]), peaks),
         "step_roofline_frac": (t_roof_attn + pb / (peaks["hbm_gbs"] * 1e9) * 1e3) / ms,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),

@@ -1,0 +1,22 @@
+"""bench.py's work counts and bounds (host arithmetic only)."""
+import pytest
+
+import bench
+from sparse_mixed_precision_b200.synth import WORKLOADS
+
+
+def test_work_counts_of_the_wan720_call():
+    w = WORKLOADS["wan720"]
+    assert bench.dense_flops(w) == pytest.approx(1.1705e14, rel=1e-3)      # 4 B H T^2 d
+    f8, f4 = bench.executed_flops(w)
+    assert (f8, f4) == (pytest.approx(1.332e13, rel=1e-3), pytest.approx(3.995e13, rel=1e-3))
+    assert bench.prep_bytes(w) == pytest.approx(4.31e9, rel=1e-2)
+    assert bench.draft_flops(w) == pytest.approx(2 * 2 * 630 ** 2 * 128 * 40)
+
+
+def test_draft_alu_bound():
+    w = WORKLOADS["wan720"]
+    assert bench.fp32_fma_peak_tflops(1965.0) == pytest.approx(148 * 128 * 2 * 1.965e9 / 1e12)
+    e = bench.draft_alu_entry(w, 1.0, {"sm_max_mhz": 1965.0})
+    assert e["bound"] == "alu" and e["frac"] == pytest.approx(e["achieved"] / e["peak"])
+    assert e["achieved"] == pytest.approx(bench.draft_flops(w) / 1e-3 / 1e12)
