@@ -92,3 +92,35 @@ def test_rank_degenerate_budgets():
     assert tags.sum() == 0 and l8.shape == (3, 0) and l4.shape == (3, 0)
     tags, l8, l4 = O.rank(sc, 7, 0)
     assert np.all(tags == 2) and np.array_equal(l8, np.tile(np.arange(7), (3, 1)))
+
+
+def test_draft_selection_tracks_true_block_mass():
+    # [DA2] Abstract: the low-resolution draft map estimates block importance. Against the
+    # true attention mass of each key block (dense fp64 softmax over the valid tokens,
+    # averaged over the query block's rows), the kept set must share far more blocks with
+    # the true top set than chance (half of them here: 32 kept of 64) would; a reversed
+    # ranking shares about a quarter.
+    w = WORKLOADS["tiny"]
+    q, k, v = generate(w, device="cpu")
+    for h in range(w.H):
+        w1 = scaled(w, B=1, H=1)
+        qh, kh, vh = (x[:, h:h + 1] for x in (q, k, v))
+        P = O.prepare(w1, qh, kh, vh)
+        sel = O.draft_select(P)
+        g = P["g"]
+        qp, kp = (O.permute(x.float().numpy(), g).astype(np.float64) for x in (qh, kh))
+        Q, K = qp[0, 0], kp[0, 0].reshape(g.N * g.bs, -1)
+        valid = np.asarray(P["valid"]).reshape(-1).astype(bool)
+        nk = g.n8 + g.n4
+        shared = []
+        for i in range(g.N):
+            S = g.sm_scale * Q[i] @ K.T
+            S[:, ~valid] = -np.inf
+            S -= S.max(axis=1, keepdims=True)
+            Pm = np.exp(S)
+            Pm /= Pm.sum(axis=1, keepdims=True)
+            mass = Pm.reshape(g.bs, g.N, g.bs).sum(axis=2).mean(axis=0)
+            top = np.argsort(-mass, kind="stable")[:nk]
+            kept = np.union1d(sel["list8"][0, 0, i], sel["list4"][0, 0, i])
+            shared.append(len(np.intersect1d(top, kept)) / nk)
+        assert np.mean(shared) >= 0.65, (h, np.mean(shared))
