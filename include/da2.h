@@ -24,8 +24,9 @@
  *
  * Conventions shared by every call
  * --------------------------------
- *  - Inputs q, k, v and the output are bf16 [B, H, T, d], d contiguous, with frame-major
- *    token order t = f*Hf*Wf + y*Wf + x.
+ *  - Inputs q, k, v and the output are bf16 [B, H, T, d] (or [B, T, H, d] with
+ *    DA2_FLAG_LAYOUT_BTHD), d contiguous, with frame-major token order
+ *    t = f*Hf*Wf + y*Wf + x.
  *  - Window (ph, pw) tiles each frame; edge windows are padded. Blocks n = f*ny*nx +
  *    (y/ph)*nx + (x/pw), slot s = (y%ph)*pw + (x%pw), ny = ceil(Hf/ph), nx = ceil(Wf/pw),
  *    N = F*ny*nx blocks of bs = ph*pw slots; padded slots hold zeros and padded keys are
