@@ -76,7 +76,14 @@ enum {
      a fused QKV projection usually leaves them) instead of [B,H,T,d]; read and written in
      place, results identical. da2_forward_host then runs unpipelined. (The pages fix no
      tensor layout.) */
-  DA2_FLAG_LAYOUT_BTHD = 4
+  DA2_FLAG_LAYOUT_BTHD = 4,
+  /* Test hook for the failure path, never needed in use: da2_attention's copy engine
+     withholds its first K/V tile, so a bounded device wait must run out. Every bounded
+     wait's limit drops from 2 s to 50 ms; the launch sets the workspace error word, stops
+     issuing, waits for its copies and tensor-core work in flight, frees its tensor memory
+     and ends (about 0.1 s); da2_get_error then returns DA2_ERR_TIMEOUT and the output is
+     undefined. */
+  DA2_FLAG_TEST_STALL = 256
 };
 
 typedef enum da2_status {
@@ -181,19 +188,23 @@ da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const voi
    device array inside the library, which every GPU that loads the library holds until
    the process exits. Configurations whose da2_workspace_size exceeds 64 MiB are rejected
    with DA2_ERR_SCRATCH_TOO_SMALL before anything is enqueued (the tiny workload and
-   single-head 480p / 720p Wan-like layers fit; a full 40-head layer does not). The first call on a
-   device looks up the array's device address (cudaGetSymbolAddress, with that device
-   current); make that first call before any stream capture. Every call on a device shares
-   the one array and leaves its contents behind; the path clears what must start at zero
-   itself. Calls that overlap on the GPU (different streams, or several host threads on
-   one device) race on the array and give wrong results: serialise them. Asynchronous on
-   `stream` like da2_forward. The built-in workspace is not exposed, so its device error
-   word cannot be read with da2_get_error. */
+   single-head 480p / 720p Wan-like layers fit; a full 40-head layer does not), and so is
+   DA2_FLAG_EXPORT_SCORES (DA2_ERR_INVALID_ARG: the scores would stay in the hidden
+   array). Every call looks up the array's device address on the current device
+   (cudaGetSymbolAddress), so an address never outlives a device reset; the first call on
+   a device also loads the library's device code there, so make it before any stream
+   capture. Every call on a device shares the one array and leaves its contents behind;
+   the path clears what must start at zero itself. Calls that overlap on the GPU
+   (different streams, or several host threads on one device) race on the array and give
+   wrong results: serialise them. Asynchronous on `stream` like da2_forward. Its device
+   error word is read with da2_get_error(NULL, 0, cfg, stream, &word). */
 da2_status da2_forward_noalloc(const da2_config* cfg, const void* q, const void* k,
                                const void* v, void* out, cudaStream_t stream);
 
 /* Reads the workspace's device error word into *word and clears it (synchronises
-   `stream`). Returns DA2_ERR_TIMEOUT if the word was non-zero. */
+   `stream`). Returns DA2_ERR_TIMEOUT if the word was non-zero. ws = NULL reads the word of
+   the built-in array of da2_forward_noalloc (cfg as given to that call; ws_bytes is
+   ignored). */
 da2_status da2_get_error(void* ws, size_t ws_bytes, const da2_config* cfg,
                          cudaStream_t stream, uint32_t* word);
 

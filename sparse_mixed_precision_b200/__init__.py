@@ -28,6 +28,7 @@ LIB_PATH = os.path.join(_HERE, "libda2.so")
 FLAG_EXPORT_SCORES = 1
 FLAG_NO_MASS_CORRECTION = 2
 FLAG_LAYOUT_BTHD = 4          # q, k, v, out token-major [B, T, H, d]
+FLAG_TEST_STALL = 256         # test hook: a bounded wait of the attention kernel runs out
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned pointer",
           4: "workspace too small", 5: "CUDA error", 6: "device error word set",
@@ -156,16 +157,18 @@ def forward_host(cfg, q_host, k_host, v_host, out_host, dq, dk, dv, dout, ws, st
 def forward_noalloc(cfg, q, k, v, out, stream=None):
     """The whole path with the library's built-in 64 MiB device scratch as workspace, for
     callers that cannot allocate device memory (see da2_forward_noalloc in include/da2.h).
-    Calls on one device must not overlap on the GPU: they share that scratch."""
+    Calls on one device must not overlap on the GPU: they share that scratch. Its device
+    error word is read with get_error(cfg, None)."""
     _check("da2_forward_noalloc", lib().da2_forward_noalloc(
         ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _stream(stream)))
 
 
 def get_error(cfg, ws, stream=None) -> int:
-    """Reads and clears the workspace's device error word (synchronises the stream)."""
+    """Reads and clears the workspace's device error word (synchronises the stream).
+    ws=None reads the word of forward_noalloc's built-in scratch."""
     word = ctypes.c_uint32()
-    st = lib().da2_get_error(_ptr(ws), ws.numel(), ctypes.byref(cfg), _stream(stream),
-                             ctypes.byref(word))
+    st = lib().da2_get_error(_ptr(ws), 0 if ws is None else ws.numel(), ctypes.byref(cfg),
+                             _stream(stream), ctypes.byref(word))
     if st not in (0, 6):
         raise DA2Error("da2_get_error", st)
     return word.value

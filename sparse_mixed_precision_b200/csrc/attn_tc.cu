@@ -130,17 +130,18 @@ __device__ __forceinline__ uint64_t gtime() {
   return t;
 }
 
-// Bounded wait, slow path: polls until the phase completes or ~2 s have passed (nothing
-// here legitimately waits that long), then records the timeout in the error word and
-// returns false. Once any wait of the launch has run out, every later wait returns at
-// once, so a broken pipeline drains quickly instead of timing out wait by wait.
-__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, uint32_t* err, bool honour_abort) {
+// Bounded wait, slow path: polls until the phase completes or `limit_ns` have passed (2 s
+// in use: nothing here legitimately waits that long), then records the timeout in the
+// error word and returns false. Once any wait of the launch has run out, every later wait
+// returns at once, so a broken pipeline drains quickly instead of timing out wait by wait.
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                           unsigned long long limit_ns, bool honour_abort) {
   const uint64_t t0 = gtime();
   while (true) {
     for (int i = 0; i < 32; ++i)
       if (tc::mbar_try_wait(bar, parity)) return true;
     if (honour_abort && (*reinterpret_cast<volatile uint32_t*>(err) & kErrWaitTimeout)) return false;
-    if (gtime() - t0 > 2000000000ull) {
+    if (gtime() - t0 > limit_ns) {
       set_error(err, kErrWaitTimeout);
       return false;
     }
@@ -148,9 +149,9 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, uint3
 }
 // Fast path inline: one non-blocking test of the phase.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint32_t* err,
-                                         bool honour_abort = true) {
+                                         unsigned long long limit_ns, bool honour_abort = true) {
   if (tc::mbar_test_wait(bar, parity)) return true;
-  return wait_bar_slow(bar, parity, err, honour_abort);
+  return wait_bar_slow(bar, parity, err, limit_ns, honour_abort);
 }
 
 __device__ __forceinline__ int block_valid_rows(const Geo& g, int n, int& hv, int& wv) {
@@ -194,10 +195,11 @@ __device__ __noinline__ void rescale_o(uint32_t taddr, float alpha) {
 template <int D, int BS>
 __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileBars* tb, uint8_t* sm, uint32_t colP,
                                               uint32_t tmem, uint32_t lane_base, uint32_t colO, int r,
-                                              float c, int ecls, uint32_t gx, int t, float& m, float& l) {
+                                              float c, int ecls, uint32_t gx, int t, float& m, float& l,
+                                              unsigned long long wait_ns) {
   constexpr int NG = BS / 16;
   constexpr int KV4 = BS < 64 ? 64 : BS;
-  wait_bar(&tb->s_full, gx & 1, w.err);
+  wait_bar(&tb->s_full, gx & 1, w.err, wait_ns);
   tc::fence_after_sync();
   uint32_t sr[BS];
 #pragma unroll
@@ -233,7 +235,7 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
   const float bias = kLog2_448 - m_new;
   // the tile's P columns (and O) are free once its previous P V has completed
   if (t > 0) {
-    wait_bar(&tb->p_free, (gx - 1) & 1, w.err);
+    wait_bar(&tb->p_free, (gx - 1) & 1, w.err, wait_ns);
     tc::fence_after_sync();
   }
   // row-sum partials: keys 4i+0/4i+1 in sA, 4i+2/4i+3 in sB
@@ -416,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       };
       bool dead = false;                // a wait ran out: issue nothing more
       int q_rounds[2] = {0, 0};         // Q tiles loaded per tile
+      const bool stall = (g.flags & DA2_FLAG_TEST_STALL) != 0;   // test hook: stage 0 never fills
       for (int k = 0; k < rounds && !dead; ++k) {
         const int nx = has_tile(k, 1) ? 2 : 1;
         int bhx[2], ix[2];
@@ -429,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           l8x[x] = w.list8 + qi * w.n8s;
           l4x[x] = w.list4 + qi * w.n4s;
           TileBars* tb = &bars->tb[x];
-          if (!wait_bar(&tb->q_empty, (k & 1) ^ 1, w.err)) { dead = true; break; }
+          if (!wait_bar(&tb->q_empty, (k & 1) ^ 1, w.err, g.wait_ns)) { dead = true; break; }
           const uint32_t qbytes = BS * D + BS * D / 2 + (uint32_t)w.sf_qk;
           uint8_t* qs = sm + x * kQBytes;
           tc::mbar_arrive_expect_tx(&tb->q_full, qbytes);
@@ -449,7 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
             const int j = list_j(l8x[x], l4x[x], t);
             const size_t kj = (size_t)bhx[x] * N + j;
             const uint32_t s = gkv % kStages, ks = gkv / kStages;
-            if (!wait_bar(&bars->kv_empty[s], (ks & 1) ^ 1, w.err)) { dead = true; break; }
+            if (stall && gkv == 0) {      // withhold the first K/V tile: its consumer's wait runs out
+              ++gkv;
+              continue;
+            }
+            if (!wait_bar(&bars->kv_empty[s], (ks & 1) ^ 1, w.err, g.wait_ns)) { dead = true; break; }
             uint8_t* st = sm + kStage0 + s * kStageBytes;
             if (fp8) {
               tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * BS * D);
@@ -471,10 +478,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       // consumed long ago; after an aborted wait they may still be in flight).
       for (uint32_t s = 0; s < (uint32_t)kStages && s < gkv; ++s) {
         const uint32_t last = s + ((gkv - 1 - s) / kStages) * kStages;
-        wait_bar(&bars->kv_full[s], (last / kStages) & 1, w.err, false);
+        wait_bar(&bars->kv_full[s], (last / kStages) & 1, w.err, g.wait_ns, false);
       }
       for (int x = 0; x < 2; ++x)
-        if (q_rounds[x] > 0) wait_bar(&bars->tb[x].q_full, (q_rounds[x] - 1) & 1, w.err, false);
+        if (q_rounds[x] > 0) wait_bar(&bars->tb[x].q_full, (q_rounds[x] - 1) & 1, w.err, g.wait_ns, false);
     }
   } else if (warp == kMmaWarp || warp == kMmaWarp + 2) {
     // ============ MMA issue: one thread per tile (warp 8: tile A, warp 10: tile B) ============
@@ -492,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         const int nx = has_tile(k, 1) ? 2 : 1;
         const uint32_t gbase = (uint32_t)k * (uint32_t)nb;   // blocks each tile had in earlier rounds
         const uint32_t kvbase = 2u * gbase;                  // K/V stages of earlier rounds (2 tiles each)
-        dead = !wait_bar(&tb->q_full, k & 1, w.err);
+        dead = !wait_bar(&tb->q_full, k & 1, w.err, g.wait_ns);
         tc::fence_after_sync();
         if (!dead && nb > n8)
           for (int kb = 0; kb < D / 64; ++kb)
@@ -502,15 +509,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         // previous owner has read its S.
         auto issue_s = [&](int t) -> bool {
           if (x == 1) {
-            if (!wait_bar(&bars->tb[0].s_free, (gbase + t) & 1, w.err)) return false;
+            if (!wait_bar(&bars->tb[0].s_free, (gbase + t) & 1, w.err, g.wait_ns)) return false;
           } else if (t > 0) {
-            if (!wait_bar(&bars->tb[nx - 1].s_free, (gbase + t - 1) & 1, w.err)) return false;
+            if (!wait_bar(&bars->tb[nx - 1].s_free, (gbase + t - 1) & 1, w.err, g.wait_ns)) return false;
           } else if (k > 0) {
-            if (!wait_bar(&bars->tb[1].s_free, (gbase - 1) & 1, w.err)) return false;
+            if (!wait_bar(&bars->tb[1].s_free, (gbase - 1) & 1, w.err, g.wait_ns)) return false;
           }
           const uint32_t seq = kvbase + (uint32_t)(nx * t + x);   // K/V stage sequence number
           const uint32_t s = seq % kStages;
-          if (!wait_bar(&bars->kv_full[s], (seq / kStages) & 1, w.err)) return false;
+          if (!wait_bar(&bars->kv_full[s], (seq / kStages) & 1, w.err, g.wait_ns)) return false;
           tc::fence_after_sync();
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
           if (t < n8) {
@@ -532,8 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         };
         // O += P V of this tile's block t
         auto issue_pv = [&](int t) -> bool {
-          if (!wait_bar(&tb->p_full, (gbase + (uint32_t)t) & 1, w.err)) return false;
-          if (t == 0 && k > 0 && !wait_bar(&tb->o_free, (k - 1) & 1, w.err)) return false;
+          if (!wait_bar(&tb->p_full, (gbase + (uint32_t)t) & 1, w.err, g.wait_ns)) return false;
+          if (t == 0 && k > 0 && !wait_bar(&tb->o_free, (k - 1) & 1, w.err, g.wait_ns)) return false;
           tc::fence_after_sync();
           const uint32_t s = (kvbase + (uint32_t)(nx * t + x)) % kStages;
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
@@ -569,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         }
       }
       tc::mma_commit(&bars->done);
-      wait_bar(&bars->done, 0, w.err, false);   // both issuers' MMAs retired before TMEM is freed
+      wait_bar(&bars->done, 0, w.err, g.wait_ns, false);   // both issuers' MMAs retired before TMEM is freed
     }
   }
   } else {
@@ -631,10 +638,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           jC = list_j(t + 65 + lane);
         }
         const int ecls = sm[kEdge + j];
-        softmax_block<D, BS>(t < n8, w, tb, sm, colP, tmem, lane_base, colO, r, c, ecls, gx, t, m, l);
+        softmax_block<D, BS>(t < n8, w, tb, sm, colP, tmem, lane_base, colO, r, c, ecls, gx, t, m, l, g.wait_ns);
       }
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
-      if (!wait_bar(&tb->o_full, k & 1, w.err)) {
+      if (!wait_bar(&tb->o_full, k & 1, w.err, g.wait_ns)) {
         dead = true;
         break;
       }

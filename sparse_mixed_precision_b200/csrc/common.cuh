@@ -18,6 +18,7 @@ struct Geo {
   float sm_scale;
   int flags;
   int bthd;   // q, k, v, out token-major [B,T,H,d] instead of [B,H,T,d]
+  unsigned long long wait_ns;   // limit of every bounded device wait (%globaltimer ns)
 };
 
 // Element offset of token t, channel 0 of head bh = b*H + h in a q/k/v/out tensor.

@@ -9,6 +9,7 @@ cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void*
                            const void* v, cudaStream_t st);
 cudaError_t launch_draft_select(const Geo& g, const Ws& w, cudaStream_t st);
 cudaError_t launch_attention_tc(const Geo& g, const Ws& w, void* out, cudaStream_t st);
+da2_status noalloc_scratch(void** ptr, size_t* bytes);   // da2_noalloc.cu
 }  // namespace da2
 
 using namespace da2;
@@ -27,7 +28,8 @@ da2_status check_config(const da2_config* c) {
     return DA2_ERR_INVALID_ARG;
   if (c->pct_fp8 < 0 || c->pct_fp4 < 0 || c->pct_fp8 + c->pct_fp4 > 100) return DA2_ERR_INVALID_ARG;
   if (!(c->sm_scale >= 0.0f) || std::isinf(c->sm_scale)) return DA2_ERR_INVALID_ARG;
-  if (c->flags & ~(DA2_FLAG_EXPORT_SCORES | DA2_FLAG_NO_MASS_CORRECTION | DA2_FLAG_LAYOUT_BTHD))
+  if (c->flags & ~(DA2_FLAG_EXPORT_SCORES | DA2_FLAG_NO_MASS_CORRECTION | DA2_FLAG_LAYOUT_BTHD |
+                   DA2_FLAG_TEST_STALL))
     return DA2_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return DA2_ERR_UNSUPPORTED;
   const long bs = (long)c->ph * c->pw;
@@ -93,6 +95,8 @@ Geo make_geo(const da2_config* c, const da2_views& v) {
   g.sm_scale = c->sm_scale > 0.0f ? c->sm_scale : 1.0f / std::sqrt((float)c->d);
   g.flags = c->flags;
   g.bthd = (c->flags & DA2_FLAG_LAYOUT_BTHD) ? 1 : 0;
+  // nothing legitimately waits near 2 s; the test hook shortens the limit to 50 ms
+  g.wait_ns = (c->flags & DA2_FLAG_TEST_STALL) ? 50000000ull : 2000000000ull;
   return g;
 }
 
@@ -329,6 +333,12 @@ da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const voi
 
 da2_status da2_get_error(void* ws, size_t ws_bytes, const da2_config* cfg, cudaStream_t stream,
                          uint32_t* word) {
+  if (!ws) {                      // the built-in scratch of da2_forward_noalloc
+    const da2_status c = check_config(cfg);
+    if (c != DA2_OK) return c;
+    const da2_status a = noalloc_scratch(&ws, &ws_bytes);
+    if (a != DA2_OK) return a;
+  }
   da2_views vw; Geo g; Ws w;
   const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
   if (s != DA2_OK) return s;

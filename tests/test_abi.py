@@ -99,3 +99,27 @@ def test_stage_calls_reject_bad_pointers_without_touching_the_device():
     assert L.da2_draft_select(ctypes.byref(cfg), ctypes.c_void_p(0x100000), n - 1, None) == 4
     assert L.da2_prepare(ctypes.byref(cfg), None, None, None, ctypes.c_void_p(0x100000), n, None) == 1
     assert L.da2_status_string(6).startswith(b"device error word")
+
+
+def test_noalloc_host_side_refusals():
+    # da2_forward_noalloc checks its arguments before it touches the device: a missing or
+    # invalid configuration, exported scores (they would stay in the hidden scratch), a
+    # workspace larger than the 64 MiB scratch, missing tensors
+    L = da2.lib()
+    p = ctypes.c_void_p(0x100000)
+    assert L.da2_forward_noalloc(None, p, p, p, p, None) == 1
+    bad = da2.config(WORKLOADS["tiny"], flags=8)
+    assert L.da2_forward_noalloc(ctypes.byref(bad), p, p, p, p, None) == 1
+    assert L.da2_forward_noalloc(ctypes.byref(da2.config(scaled(WORKLOADS["tiny"], d=96))),
+                                 p, p, p, p, None) == 2
+    sc = da2.config(WORKLOADS["tiny"], flags=da2.FLAG_EXPORT_SCORES)
+    assert L.da2_forward_noalloc(ctypes.byref(sc), p, p, p, p, None) == 1
+    big = da2.config(WORKLOADS["wan720"])                       # about 2.2 GB of workspace
+    assert da2.workspace_size(big) > 64 << 20
+    assert L.da2_forward_noalloc(ctypes.byref(big), p, p, p, p, None) == 7
+    tiny = da2.config(WORKLOADS["tiny"])
+    assert L.da2_forward_noalloc(ctypes.byref(tiny), None, p, p, p, None) == 1
+    assert L.da2_forward_noalloc(ctypes.byref(tiny), p, p, p, None, None) == 1
+    # reading the scratch's error word needs a valid configuration first
+    word = ctypes.c_uint32()
+    assert L.da2_get_error(None, 0, ctypes.byref(bad), None, ctypes.byref(word)) == 1

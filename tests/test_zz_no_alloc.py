@@ -40,6 +40,7 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
             out = torch.full_like(q, float("nan"))
             da2.forward_noalloc(cfg, q, k, v, out)
             torch.cuda.synchronize()
+            assert da2.get_error(cfg, None) == 0, (name, call)   # the scratch's error word
             o = out.float()
             assert torch.isfinite(o).all(), (name, call)
             err = (o - ref).abs().max().item()
@@ -56,3 +57,27 @@ def test_noalloc_refuses_a_workspace_larger_than_its_scratch():
                                        ctypes.c_void_p(q.data_ptr()), None)
     assert st == 7
     assert b"64 MiB" in da2.lib().da2_status_string(7)
+
+
+def test_noalloc_reports_a_wait_that_ran_out():
+    # the built-in scratch's error word is readable: a call whose bounded wait must run out
+    # (test-only flag) reports DA2_ERR_TIMEOUT through da2_get_error(NULL, ...); the next
+    # normal call is again equal to da2_forward's output
+    w = WORKLOADS["tiny"]
+    q, k, v = generate(w, device="cuda")
+    ref = _reference(w, q, k, v)
+    out = torch.empty_like(q)
+    cfg_stall = da2.config(w, flags=da2.FLAG_TEST_STALL)
+    da2.forward_noalloc(cfg_stall, q, k, v, out)
+    torch.cuda.synchronize()
+    word = ctypes.c_uint32()
+    st = da2.lib().da2_get_error(None, 0, ctypes.byref(cfg_stall),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream),
+                                 ctypes.byref(word))
+    assert st == 6 and (word.value & 1), (st, word.value)
+    cfg = da2.config(w)
+    da2.forward_noalloc(cfg, q, k, v, out)
+    torch.cuda.synchronize()
+    assert da2.get_error(cfg, None) == 0
+    o = out.float()
+    assert (o - ref).abs().max().item() <= ATOL and ((o - ref).norm() / ref.norm()).item() <= RTOL_L2
