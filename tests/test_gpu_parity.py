@@ -255,6 +255,19 @@ def test_token_major_layout_matches(name, heads):
     assert da2.get_error(cfg, ws) == 0 and da2.get_error(cfg_t, ws_t) == 0
     assert torch.equal(ws, ws_t)
     assert torch.equal(out_t.transpose(1, 2), out)
+    # and against the oracle directly: the token-major output, read back per head, on the
+    # selection the token-major call made
+    rd = WsReader(ws_t, da2.workspace_views(cfg_t), w.d)
+    g = O.geometry(scaled(w, B=1, H=1))
+    rng = np.random.default_rng(3)
+    edge = [i for i in range(g.N) if O.block_counts(g)[i] < g.bs]
+    for h in sorted({0, w.H - 1}):
+        qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+        P = check_prep(w, da2.workspace_views(cfg_t), rd, h, qh, kh, vh)
+        l8, l4 = rd.lists(h, h + 1)
+        blocks = list(range(g.N)) if g.N <= 64 else sorted(set(
+            [0, g.N - 1] + list(rng.choice(g.N, 4, replace=False)) + list(rng.choice(edge, 2, replace=False))))
+        check_attention(w, None, P, l8[0], l4[0], out_t[0, :, h].float().cpu().numpy(), blocks, g)
     # the host-buffer path takes the same layout (unpipelined)
     oh = torch.empty(qt.shape, dtype=qt.dtype).pin_memory()
     dq, dk, dv, dout = (torch.empty_like(qt) for _ in range(4))
