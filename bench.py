@@ -102,6 +102,33 @@ def attention_traffic(w):
     return rec["attention_dram_bytes"] * (w.B * w.H) / rec["captured_bh"]
 
 
+def draft_bytes(w) -> float:
+    """Algorithmic HBM bytes of the draft stage: reads the four pooled fp32 [N, d] arrays
+    per head, writes the u8 tags [N, N] and the i16 lists [N, n8] + [N, n4] per head."""
+    import math as _m
+    N = w.F * _m.ceil(w.Hf / w.ph) * _m.ceil(w.Wf / w.pw)
+    n8 = (w.pct_fp8 * N + 50) // 100
+    n4 = ((w.pct_fp8 + w.pct_fp4) * N + 50) // 100 - n8
+    BH = w.B * w.H
+    return float(BH * (4 * N * w.d * 4 + N * N + N * (max(n8, 1) + max(n4, 1)) * 2))
+
+
+def hbm_entry(bytes_: float, ms: float, peaks: dict) -> dict:
+    gbs = bytes_ / (ms * 1e-3) / 1e9
+    return {"achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+            "bytes": bytes_}
+
+
+def tensor_roofline_ms(w, peaks: dict, sustained: bool = False) -> float:
+    """Precision-weighted tensor-core time of the executed FP8 and FP4 work: FP8 at 2x and
+    FP4 at 4x the measured bf16 rate (NVIDIA's nominal dense ratios 2.25 : 4.5 : 9 PFLOP/s).
+    The burst bf16 figure fits a kernel timed alone; the sustained one a long loop at the
+    power cap."""
+    bf16 = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops", peaks.get("bf16_tflops"))
+    f8, f4 = executed_flops(w)
+    return (f8 / (2.0 * bf16 * 1e12) + f4 / (4.0 * bf16 * 1e12)) * 1e3
+
+
 def draft_alu_entry(w, draft_ms: float, peaks: dict) -> dict:
     """The draft stage against its own bound: fp32 FMA throughput (ALU-bound; it reads only
     the 52 MB of pooled vectors), peak from the unit counts at the measured max SM clock."""
@@ -238,6 +265,8 @@ def oracle_sample(w, q, k, v, n_blocks: int):
     from sparse_mixed_precision_b200.synth import scaled
     wh = scaled(w, B=1, H=1)
     qh, kh, vh = (x[:1, :1].cpu() for x in (q, k, v))
+    from threadpoolctl import threadpool_limits
+    limiter = threadpool_limits(1)        # the oracle runs on one host thread
     t0 = time.perf_counter()
     P = O.prepare(wh, qh, kh, vh)
     sel = O.draft_select(P)
@@ -248,11 +277,13 @@ def oracle_sample(w, q, k, v, n_blocks: int):
     t2 = time.perf_counter()
     O.attention(ops, P["valid"], sel["list8"], sel["list4"], g.sm_scale, True, blocks=blocks)
     t3 = time.perf_counter()
+    limiter.unregister() if hasattr(limiter, "unregister") else limiter.restore_original_limits()
     per_head = (t1 - t0) + (t3 - t2) * g.N / len(blocks)
     sec = per_head * w.B * w.H
     desc = (f"oracle on head (0,0): prepare+select {t1 - t0:.2f} s, attention of {len(blocks)}"
             f" of {g.N} query blocks {t3 - t2:.2f} s; extrapolated x{g.N / len(blocks):.1f}"
-            f" blocks and x{w.B * w.H} heads")
+            f" blocks and x{w.B * w.H} heads; one host thread (BLAS limited to 1) of"
+            f" {os.cpu_count()} on the host")
     return sec, desc
 
 
@@ -278,7 +309,7 @@ def run_reference(args, w, ws_size, rank):
             per_step.append(sec)
     sec = statistics.mean(per_step)
     value = dense_flops(w) / sec / 1e12
-    cores = blas_threads()
+    cores = 1
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -299,6 +330,79 @@ def config_dict(w, args):
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
 
 
+def time_stages(da2, w, q, k, v, steps, warmup, dev, flush, clocks=None):
+    """Runs `warmup` untimed and `steps` timed calls (prepare, draft_select, attention on one
+    stream, L2 flushed before each) and returns the per-stage CUDA-event times (ms lists),
+    the workspace and the output of the last call."""
+    cfg = da2.config(w)
+    ws = torch.empty(da2.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        da2.prepare(cfg, q, k, v, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        da2.draft_select(cfg, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        da2.attention(cfg, ws, out, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert da2.get_error(cfg, ws) == 0
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.__enter__()
+    for s_ in range(steps):
+        flush.zero_()
+        step(events[s_])
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.__exit__(None, None, None)
+    assert da2.get_error(cfg, ws) == 0
+    stage = {"prepare": [], "draft_select": [], "attention": [], "total": []}
+    for ev in events:
+        stage["prepare"].append(ev[0].elapsed_time(ev[1]))
+        stage["draft_select"].append(ev[1].elapsed_time(ev[2]))
+        stage["attention"].append(ev[2].elapsed_time(ev[3]))
+        stage["total"].append(ev[0].elapsed_time(ev[3]))
+    return stage, cfg, ws, out
+
+
+def dense_rel_l2(q, k, v, out, heads, rows=4096, seed=0):
+    """Relative L2 error of the call's output against dense fp32 softmax attention (torch
+    on the GPU, a reference computation), on `rows` seeded query rows of each listed head."""
+    g = torch.Generator().manual_seed(seed)
+    res = {}
+    for b, h in heads:
+        r = torch.randperm(q.shape[2], generator=g)[:rows].to(q.device)
+        S = (q[b, h, r].float() @ k[b, h].float().T) / math.sqrt(q.shape[-1])
+        ref = torch.softmax(S, -1) @ v[b, h].float()
+        got = out[b, h, r].float()
+        res[f"b{b}h{h}"] = ((got - ref).norm() / ref.norm()).item()
+    return res
+
+
+def workload_entry(w, stage, peaks):
+    """ms, dense-equivalent TFLOP/s and roofline fractions of one workload's call."""
+    ms = statistics.mean(stage["total"])
+    attn = statistics.mean(stage["attention"])
+    t8 = tensor_roofline_ms(w, peaks)
+    return {"ms": ms, "tflops": dense_flops(w) / (ms * 1e-3) / 1e12,
+            "stages_ms": {k_: statistics.mean(v_) for k_, v_ in stage.items() if k_ != "total"},
+            "attention_frac": t8 / attn, "t_roof_attention_ms": t8,
+            "prepare_hbm_frac": prep_bytes(w) / (statistics.mean(stage["prepare"]) * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "draft_hbm_frac": draft_bytes(w) / (statistics.mean(stage["draft_select"]) * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -311,6 +415,8 @@ def main():
                     help="override the head count (small cases for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload lines (the other configurations)")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     if args.heads > 0:
@@ -328,85 +434,55 @@ def main():
     import sparse_mixed_precision_b200 as da2
     dev = torch.device("cuda", local)
     q, k, v = generate(w, device=dev, seed=w.seed + rank)
-    cfg = da2.config(w)
-    views = da2.workspace_views(cfg)
-    ws = torch.empty(views["total"], dtype=torch.uint8, device=dev)
-    out = torch.empty_like(q)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        da2.prepare(cfg, q, k, v, ws, stream)
-        if ev is not None:
-            ev[1].record(stream)
-        da2.draft_select(cfg, ws, stream)
-        if ev is not None:
-            ev[2].record(stream)
-        da2.attention(cfg, ws, out, stream)
-        if ev is not None:
-            ev[3].record(stream)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    assert da2.get_error(cfg, ws) == 0
-
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for s in range(args.steps):
-            flush.zero_()
-            step(events[s])
-        torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    stage, cfg, ws, out = time_stages(da2, w, q, k, v, args.steps, args.warmup, dev, flush, clocks=clk)
     barrier(world)
-    stage = {"prepare": [], "draft_select": [], "attention": []}
-    total = []
-    for ev in events:
-        a, b, c, d = (ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
-                      ev[2].elapsed_time(ev[3]), ev[0].elapsed_time(ev[3]))
-        stage["prepare"].append(a)
-        stage["draft_select"].append(b)
-        stage["attention"].append(c)
-        total.append(d)
-    ms_local = sum(total) / len(total)
+    ms_local = statistics.mean(stage["total"])
     ms = max_over_ranks(ms_local, world)
-    assert da2.get_error(cfg, ws) == 0
     value = job_throughput(w, world, ms)
 
-    # roofline of the dominant kernel (attention): precision-weighted tensor bound
+    # roofline of the dominant kernel (attention): precision-weighted tensor bound, against
+    # the burst bf16 figure (the kernel is timed alone, one call at a time) and, beside it,
+    # the sustained one
     peaks, src = load_peaks()
-    bf16 = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    p8, p4 = 2.0 * bf16, 4.0 * bf16          # nominal dense ratios fp8 : fp4 : bf16 = 2 : 4 : 1
     f8, f4 = executed_flops(w)
     attn_ms = statistics.mean(stage["attention"])
-    t_roof_attn = (f8 / (p8 * 1e12) + f4 / (p4 * 1e12)) * 1e3
+    t_roof = tensor_roofline_ms(w, peaks)
+    t_roof_sus = tensor_roofline_ms(w, peaks, sustained=True)
     achieved = (f8 + f4) / (attn_ms * 1e-3) / 1e12
-    peak_eff = (f8 + f4) / (t_roof_attn * 1e-3) / 1e12
+    peak_eff = (f8 + f4) / (t_roof * 1e-3) / 1e12
     prep_ms = statistics.mean(stage["prepare"])
-    pb = prep_bytes(w)
+    draft_ms = statistics.mean(stage["draft_select"])
+    pb, db = prep_bytes(w), draft_bytes(w)
     traffic = attention_traffic(w)
+    bf16 = peaks.get("bf16_tflops")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3/e2m1 MMA, f32 accumulate", "data": "synthetic (seeded smooth field + noise + sinks)",
         "config": config_dict(w, args),
-        "stages_ms": {k_: statistics.mean(v_) for k_, v_ in stage.items()},
+        "stages_ms": {k_: statistics.mean(v_) for k_, v_ in stage.items() if k_ != "total"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff, "unit": "TFLOP/s",
-                     "frac": t_roof_attn / attn_ms, "traffic": traffic,
+                     "frac": t_roof / attn_ms, "traffic": traffic,
+                     "frac_sustained_peak": t_roof_sus / attn_ms,
                      "note": f"attention kernel; peak = precision-weighted ({f8:.3e} FP8 + {f4:.3e} FP4 FLOP"
-                             f" at {p8:.0f} / {p4:.0f} TFLOP/s = 2x / 4x {src} sustained bf16)"},
-        "prepare_hbm": {"achieved_gbs": pb / (prep_ms * 1e-3) / 1e9, "peak_gbs": peaks["hbm_gbs"],
-                        "frac": pb / (prep_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-        "draft_alu": draft_alu_entry(w, statistics.mean(stage["draft_select"]), peaks),
-        "step_roofline_frac": (t_roof_attn + pb / (peaks["hbm_gbs"] * 1e9) * 1e3) / ms,
+                             f" at {2 * bf16:.0f} / {4 * bf16:.0f} TFLOP/s = 2x / 4x the {src} burst bf16"
+                             f" cuBLAS rate, t_roof {t_roof:.2f} ms; frac_sustained_peak uses the"
+                             f" sustained bf16 rate, t_roof {t_roof_sus:.2f} ms)"},
+        "prepare_hbm": hbm_entry(pb, prep_ms, peaks),
+        "draft_hbm": hbm_entry(db, draft_ms, peaks),
+        "draft_alu": draft_alu_entry(w, draft_ms, peaks),
+        "step_roofline_frac": (t_roof + (pb + db) / (peaks["hbm_gbs"] * 1e9) * 1e3) / ms,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }
+    if rank == 0 and args.heads == 0:
+        line["dense_rel_l2"] = dense_rel_l2(q, k, v, out, [(0, 0), (w.B - 1, w.H - 1)])
 
     # end to end through the C ABI with host buffers (pinned), copies inside the timed region
     if not args.no_e2e:
@@ -427,11 +503,28 @@ def main():
         line["e2e"] = {"value": job_throughput(w, world, e2e_ms), "unit": UNIT,
                        "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * nbytes,
                        "d2h_bytes_per_step": nbytes}
+        del qh, kh, vh, oh
+
+    # the other configurations: per-workload ms, TFLOP/s and roofline fractions (the
+    # headline value above stays on the 720p layer); rank 0 of a single-GPU run only
+    if rank == 0 and world == 1 and not args.no_workloads and args.heads == 0:
+        del ws, out
+        others = {}
+        for name in ("wan480", "hunyuan720", "sweep0", "sweep1", "sweep2", "sweep3", "sweep4"):
+            if name == w.name:
+                continue
+            wo = WORKLOADS[name]
+            qo, ko, vo = generate(wo, device=dev)
+            st, _, wso, oo = time_stages(da2, wo, qo, ko, vo, 5, 3, dev, flush)
+            others[name] = workload_entry(wo, st, peaks)
+            del qo, ko, vo, wso, oo
+            torch.cuda.empty_cache()
+        line["workloads"] = others
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sec, desc = oracle_sample(w, q, k, v, args.ref_blocks)
         line["cpu_baseline"] = {"value": dense_flops(w) / sec / 1e12, "unit": UNIT,
-                                "cores": blas_threads(), "kind": "oracle", "sample": desc,
+                                "cores": 1, "kind": "oracle", "sample": desc,
                                 "ms_per_call": sec * 1e3}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -20,3 +20,15 @@ def test_draft_alu_bound():
     e = bench.draft_alu_entry(w, 1.0, {"sm_max_mhz": 1965.0})
     assert e["bound"] == "alu" and e["frac"] == pytest.approx(e["achieved"] / e["peak"])
     assert e["achieved"] == pytest.approx(bench.draft_flops(w) / 1e-3 / 1e12)
+
+
+def test_draft_bytes_and_tensor_roofline():
+    w = WORKLOADS["wan720"]
+    # pooled fp32 [N, d] x 4 read, u8 tags [N, N] and i16 lists [N, 63 + 189] written, 40 heads
+    assert bench.draft_bytes(w) == pytest.approx(40 * (4 * 630 * 128 * 4 + 630 * 630 + 630 * 252 * 2))
+    peaks = {"bf16_tflops": 1655.5, "bf16_tflops_sustained": 1405.2}
+    f8, f4 = bench.executed_flops(w)
+    assert bench.tensor_roofline_ms(w, peaks) == pytest.approx(
+        (f8 / 3311e12 + f4 / 6622e12) * 1e3)                      # 10.06 ms at the burst rate
+    assert bench.tensor_roofline_ms(w, peaks) == pytest.approx(10.06, rel=2e-3)
+    assert bench.tensor_roofline_ms(w, peaks, sustained=True) > bench.tensor_roofline_ms(w, peaks)
