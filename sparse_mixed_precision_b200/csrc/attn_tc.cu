@@ -233,19 +233,23 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
   const float m_new = fmaxf(m, mh * c);
   const float alpha = ex2(m - m_new);
   const float bias = kLog2_448 - m_new;
-  // the tile's P columns (and O) are free once its previous P V has completed
-  if (t > 0) {
-    wait_bar(&tb->p_free, (gx - 1) & 1, w.err, wait_ns);
-    tc::fence_after_sync();
-  }
+  // The quantised P stays in registers until the exponential loop is done: only then does
+  // the row wait for its tile's previous P V (which frees the P columns and O), so that
+  // wait overlaps the loop.
+  auto wait_p_free = [&]() {
+    if (t > 0) {
+      wait_bar(&tb->p_free, (gx - 1) & 1, w.err, wait_ns);
+      tc::fence_after_sync();
+    }
+  };
   // row-sum partials: keys 4i+0/4i+1 in sA, 4i+2/4i+3 in sB
   f32x2 sA = pk2(0.0f, 0.0f), sB = pk2(0.0f, 0.0f);
   const f32x2 c2 = pk2(c, c);
   if (FP8) {
     const f32x2 b2 = pk2(bias, bias);
+    uint32_t wd[BS / 4];
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
-      uint32_t wd[4];
 #pragma unroll
       for (int e = 0; e < 16; e += 4) {
         float x0, x1, x2, x3;
@@ -254,10 +258,12 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
         const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
         sA = add2(sA, pk2(p0, p1));
         sB = add2(sB, pk2(p2, p3));
-        wd[e / 4] = (uint32_t)f32x2_to_e4m3x2(p0, p1) | ((uint32_t)f32x2_to_e4m3x2(p2, p3) << 16);
+        wd[4 * q + e / 4] = (uint32_t)f32x2_to_e4m3x2(p0, p1) | ((uint32_t)f32x2_to_e4m3x2(p2, p3) << 16);
       }
-      tc::tmem_st4(tmem + lane_base + colP + 4 * q, wd);
     }
+    wait_p_free();
+#pragma unroll
+    for (int q = 0; q < NG; ++q) tc::tmem_st4(tmem + lane_base + colP + 4 * q, wd + 4 * q);
   } else {
     uint32_t sfw[KV4 / 64];
 #pragma unroll
@@ -283,6 +289,7 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
       gs[q + 1] = sg.y > 0.0f ? sg.y : 1.0f;
       sfw[q >> 2] |= sc2 << (8 * (q & 3));
     }
+    uint32_t pw[2 * NG];
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
       const f32x2 b2 = pk2(gb[q], gb[q]);
@@ -306,8 +313,12 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
       const float gsum = (a0 + a1) + (b0 + b1);
       if (q & 1) sB = add2(sB, pk2(gs[q] * gsum, 0.0f));
       else sA = add2(sA, pk2(gs[q] * gsum, 0.0f));
-      tc::tmem_st2(tmem + lane_base + colP + 2 * q, f32x8_to_e2m1x8(y), f32x8_to_e2m1x8(y + 8));
+      pw[2 * q] = f32x8_to_e2m1x8(y);
+      pw[2 * q + 1] = f32x8_to_e2m1x8(y + 8);
     }
+    wait_p_free();
+#pragma unroll
+    for (int q = 0; q < NG; q += 2) tc::tmem_st4(tmem + lane_base + colP + 2 * q, pw + 2 * q);
 #pragma unroll
     for (int gk = BS; gk < KV4; gk += 16)                  // zero keys past the block (32-token blocks)
       tc::tmem_st2(tmem + lane_base + colP + gk / 8, 0u, 0u);
