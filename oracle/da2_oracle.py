@@ -34,7 +34,7 @@ import numpy as np
 F32 = np.float32
 E4M3_MAX = 448.0        # largest finite E4M3 value (OCP FP8, bias 7, no infinities)
 E2M1_MAX = 6.0          # largest E2M1 value
-TAG_SKIP, TAG_FP4, TAG_FP8 = 0, 1, 2
+TAG_SKIP, TAG_FP4, TAG_FP8, TAG_MIX = 0, 1, 2, 3
 
 
 # ----------------------------------------------------------------------------------------
@@ -59,6 +59,7 @@ class Geometry:
     n8: int       # FP8 blocks per query block
     n4: int       # FP4 blocks per query block
     sm_scale: float
+    nm: int = 0   # mixed blocks per query block (E4M3 scores, E2M1 P V)
 
 
 def budget_counts(N: int, pct_fp8: int, pct_fp4: int) -> tuple[int, int]:
@@ -73,14 +74,29 @@ def budget_counts(N: int, pct_fp8: int, pct_fp4: int) -> tuple[int, int]:
     return n8, nk - n8
 
 
+def budget_counts3(N: int, pct_fp8: int, pct_mix: int, pct_fp4: int) -> tuple[int, int, int]:
+    """Blocks kept at FP8, mixed and FP4 per query block: the three classes take the
+    ranking's top blocks in that order, each cumulative cut rounded half up as in
+    `budget_counts` (with pct_mix = 0 the FP8 and FP4 counts are those of `budget_counts`).
+
+    [DA2] Abstract: the shared ranking gives higher precision to the more important
+    blocks and lower precision to the rest under configurable budgets; the mixed class
+    (8-bit scores, 4-bit probabilities and values) is a precision between the two.
+    """
+    c8 = (pct_fp8 * N + 50) // 100
+    c8m = ((pct_fp8 + pct_mix) * N + 50) // 100
+    ck = ((pct_fp8 + pct_mix + pct_fp4) * N + 50) // 100
+    return c8, c8m - c8, ck - c8m
+
+
 def geometry(w) -> Geometry:
     ny, nx = -(-w.Hf // w.ph), -(-w.Wf // w.pw)
     N = w.F * ny * nx
     bs = w.ph * w.pw
-    n8, n4 = budget_counts(N, w.pct_fp8, w.pct_fp4)
+    n8, nm, n4 = budget_counts3(N, w.pct_fp8, getattr(w, "pct_mix", 0), w.pct_fp4)
     sm = getattr(w, "sm_scale", 0.0) or 1.0 / math.sqrt(w.d)
     return Geometry(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, ny, nx, N, bs,
-                    w.F * w.Hf * w.Wf, N * bs, n8, n4, sm)
+                    w.F * w.Hf * w.Wf, N * bs, n8, n4, sm, nm)
 
 
 def token_block_slot(g: Geometry):
@@ -330,12 +346,12 @@ def draft_scores(qavg, kavg, qmax, kmax, counts, sm_scale, mass_correction=True)
     return 0.5 * (one(qavg, kavg) + one(qmax, kmax))
 
 
-def rank(scores, n8: int, n4: int):
-    """Shared ranking of each row: order (score desc, block index asc); the first n8 blocks
-    are FP8, the next n4 FP4, the rest skipped.
+def rank_classes(scores, n8: int, nm: int, n4: int):
+    """Shared ranking of each row into four classes: order (score desc, block index asc);
+    the first n8 blocks are FP8, the next nm mixed, the next n4 FP4, the rest skipped.
 
-    Returns tags uint8 [..., N, N] (0 skip, 1 FP4, 2 FP8), list8 int [..., N, n8] and
-    list4 int [..., N, n4], each list in ascending block index.
+    Returns tags uint8 [..., N, N] (0 skip, 1 FP4, 2 FP8, 3 mixed) and the ascending block
+    lists of each kept class: list8 [..., N, n8], listm [..., N, nm], list4 [..., N, n4].
     """
     sc = np.asarray(scores)
     lead = sc.shape[:-1]
@@ -343,15 +359,23 @@ def rank(scores, n8: int, n4: int):
     flat = sc.reshape(-1, N)
     j = np.arange(N)
     tags = np.zeros(flat.shape, dtype=np.uint8)
-    l8 = np.zeros((flat.shape[0], n8), dtype=np.int64)
-    l4 = np.zeros((flat.shape[0], n4), dtype=np.int64)
+    cuts = ((TAG_FP8, 0, n8), (TAG_MIX, n8, n8 + nm), (TAG_FP4, n8 + nm, n8 + nm + n4))
+    lists = {t: np.zeros((flat.shape[0], b - a), dtype=np.int64) for t, a, b in cuts}
     for r in range(flat.shape[0]):
         order = np.lexsort((j, -flat[r]))
-        tags[r, order[:n8]] = TAG_FP8
-        tags[r, order[n8:n8 + n4]] = TAG_FP4
-        l8[r] = np.sort(order[:n8])
-        l4[r] = np.sort(order[n8:n8 + n4])
-    return (tags.reshape(lead + (N,)), l8.reshape(lead + (n8,)), l4.reshape(lead + (n4,)))
+        for t, a, b in cuts:
+            tags[r, order[a:b]] = t
+            lists[t][r] = np.sort(order[a:b])
+    return dict(tags=tags.reshape(lead + (N,)),
+                list8=lists[TAG_FP8].reshape(lead + (n8,)),
+                listm=lists[TAG_MIX].reshape(lead + (nm,)),
+                list4=lists[TAG_FP4].reshape(lead + (n4,)))
+
+
+def rank(scores, n8: int, n4: int):
+    """The two-class ranking (no mixed blocks): tags, list8 and list4 of `rank_classes`."""
+    r = rank_classes(scores, n8, 0, n4)
+    return r["tags"], r["list8"], r["list4"]
 
 
 # ----------------------------------------------------------------------------------------
@@ -396,11 +420,13 @@ def operands_exact(qp, kp, vp) -> Operands:
 
 
 def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
-              return_parts=False, blocks=None):
-    """Block-sparse attention with one online softmax over both phases.
+              return_parts=False, blocks=None, listm=None):
+    """Block-sparse attention with one online softmax over all phases.
 
     For each (b, h, query block i): the FP8 phase visits list8[i] in ascending block index,
-    then the FP4 phase visits list4[i]; each visited block j updates the running row max
+    then the mixed phase visits listm[i] (scores from the E4M3 copies of Q and K, P
+    quantised as for FP4 and multiplied with the E2M1 copy of V), then the FP4 phase visits
+    list4[i]; each visited block j updates the running row max
     m, rescales the running sum l and accumulator by exp(m_old - m_new), adds
     sum(exp(S - m_new)) to l (unquantised) and adds P~ V to the accumulator, with P~ the
     block's quantised probabilities taken against the running max. Padded key slots are
@@ -421,7 +447,11 @@ def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
                 l = np.zeros(bs)
                 acc = np.zeros((bs, d))
                 rec = []
-                for prec, lst in ((8, list8[b, h, i]), (4, list4[b, h, i])):
+                phases = [(8, 8, list8[b, h, i])]
+                if listm is not None:
+                    phases.append((8, 4, listm[b, h, i]))
+                phases.append((4, 4, list4[b, h, i]))
+                for prec, pprec, lst in phases:       # score precision, P V precision
                     qi = ops.q[prec][b, h, i]
                     for j in lst:
                         S = sm_scale * (qi @ ops.k[prec][b, h, j].T)
@@ -431,8 +461,8 @@ def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
                         alpha = np.where(np.isfinite(m), np.exp(m - np.where(fin, m_new, 0.0)), 0.0)
                         p = np.exp(S - np.where(fin, m_new, 0.0)[:, None])
                         p[~np.isfinite(S)] = 0.0
-                        pq = quant_p(p, prec) if quantise_p else p
-                        pv = pq @ ops.v[prec][b, h, j]
+                        pq = quant_p(p, pprec) if quantise_p else p
+                        pv = pq @ ops.v[pprec][b, h, j]
                         l = alpha * l + p.sum(axis=1)
                         acc = alpha[:, None] * acc + pv
                         if return_parts:
@@ -547,23 +577,29 @@ def draft_select(prep, mass_correction=True):
     g = prep["g"]
     sc = draft_scores(prep["qavg"], prep["kavg"], prep["qmax"], prep["kmax"],
                       prep["counts"], g.sm_scale, mass_correction)
-    tags, l8, l4 = rank(sc, g.n8, g.n4)
-    return dict(scores=sc, tags=tags, list8=l8, list4=l4)
+    r = rank_classes(sc, g.n8, g.nm, g.n4)
+    return dict(scores=sc, **r)
 
 
 def run(w, q, k, v, quantised=True, lists=None):
     """Whole hot path. Returns dict with every intermediate and `out` fp64 [B,H,T,d].
 
-    `lists` = (list8, list4) overrides the oracle's own selection (used to compare the
-    attention step on the CUDA path's selection when rankings differ at near-ties).
+    `lists` = (list8, list4) or (list8, list4, listm) overrides the oracle's own selection
+    (used to compare the attention step on the CUDA path's selection when rankings differ
+    at near-ties).
     """
     prep = prepare(w, q, k, v)
     g = prep["g"]
     sel = draft_select(prep)
-    l8, l4 = (sel["list8"], sel["list4"]) if lists is None else lists
+    if lists is None:
+        l8, l4, lm = sel["list8"], sel["list4"], sel["listm"]
+    else:
+        l8, l4 = lists[0], lists[1]
+        lm = lists[2] if len(lists) > 2 else None
     if quantised:
         ops = operands_quantised(prep["Q"], prep["K"], prep["V"])
     else:
         ops = operands_exact(prep["qp"], prep["kp"], prep["vp"])
-    o = attention(ops, prep["valid"], l8, l4, g.sm_scale, quantise_p=quantised)
+    o = attention(ops, prep["valid"], l8, l4, g.sm_scale, quantise_p=quantised,
+                  listm=lm if (lm is not None and lm.shape[-1] > 0) else None)
     return dict(prep=prep, sel=sel, out_blocks=o, out=inverse_permute(o, g))

@@ -40,6 +40,7 @@ class Workload:
     sinks: int = 0
     temperature: bool = False
     seed: int = 0
+    pct_mix: int = 0     # percent of KV blocks with E4M3 scores and E2M1 P V (between FP8 and FP4)
 
     @property
     def T(self) -> int:
