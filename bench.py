@@ -37,16 +37,20 @@ def dense_flops(w) -> float:
 
 
 def executed_flops(w):
-    """(FP8, FP4) tensor FLOPs actually executed: kept block pairs x 4 bs^2 d."""
+    """(FP8, FP4) tensor FLOPs actually executed: kept block pairs x 4 bs^2 d (half of it
+    Q K^T, half P V); a mixed block's Q K^T counts as FP8 and its P V as FP4."""
     import math as _m
     ny, nx = _m.ceil(w.Hf / w.ph), _m.ceil(w.Wf / w.pw)
     N = w.F * ny * nx
     bs = w.ph * w.pw
-    n8 = (w.pct_fp8 * N + 50) // 100
-    nk = ((w.pct_fp8 + w.pct_fp4) * N + 50) // 100
+    pm = getattr(w, "pct_mix", 0)
+    c8 = (w.pct_fp8 * N + 50) // 100
+    c8m = ((w.pct_fp8 + pm) * N + 50) // 100
+    ck = ((w.pct_fp8 + pm + w.pct_fp4) * N + 50) // 100
     rows = w.B * w.H * N
     per = 4.0 * bs * bs * w.d
-    return rows * n8 * per, rows * (nk - n8) * per
+    nm = c8m - c8
+    return rows * (c8 + 0.5 * nm) * per, rows * (ck - c8m + 0.5 * nm) * per
 
 
 def draft_flops(w) -> float:
@@ -104,13 +108,16 @@ def attention_traffic(w):
 
 def draft_bytes(w) -> float:
     """Algorithmic HBM bytes of the draft stage: reads the four pooled fp32 [N, d] arrays
-    per head, writes the u8 tags [N, N] and the i16 lists [N, n8] + [N, n4] per head."""
+    per head, writes the u8 tags [N, N] and the i16 lists of the kept classes per head."""
     import math as _m
     N = w.F * _m.ceil(w.Hf / w.ph) * _m.ceil(w.Wf / w.pw)
-    n8 = (w.pct_fp8 * N + 50) // 100
-    n4 = ((w.pct_fp8 + w.pct_fp4) * N + 50) // 100 - n8
+    pm = getattr(w, "pct_mix", 0)
+    c8 = (w.pct_fp8 * N + 50) // 100
+    c8m = ((w.pct_fp8 + pm) * N + 50) // 100
+    ck = ((w.pct_fp8 + pm + w.pct_fp4) * N + 50) // 100
+    kept = max(c8, 1) + max(ck - c8m, 1) + (c8m - c8 if pm > 0 else 0)
     BH = w.B * w.H
-    return float(BH * (4 * N * w.d * 4 + N * N + N * (max(n8, 1) + max(n4, 1)) * 2))
+    return float(BH * (4 * N * w.d * 4 + N * N + N * kept * 2))
 
 
 def hbm_entry(bytes_: float, ms: float, peaks: dict) -> dict:
@@ -510,7 +517,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_workloads and args.heads == 0:
         del ws, out
         others = {}
-        for name in ("wan480", "hunyuan720", "sweep0", "sweep1", "sweep2", "sweep3", "sweep4"):
+        for name in ("wan480", "hunyuan720", "sweep0", "sweep1", "sweep2", "sweep3", "sweep4", "wan720mix"):
             if name == w.name:
                 continue
             wo = WORKLOADS[name]

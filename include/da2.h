@@ -31,17 +31,21 @@
  *    (y/ph)*nx + (x/pw), slot s = (y%ph)*pw + (x%pw), ny = ceil(Hf/ph), nx = ceil(Wf/pw),
  *    N = F*ny*nx blocks of bs = ph*pw slots; padded slots hold zeros and padded keys are
  *    masked out of the attention.
- *  - Budgets: n8 = floor((pct_fp8*N + 50)/100) FP8 KV blocks and n4 = floor(((pct_fp8 +
- *    pct_fp4)*N + 50)/100) - n8 FP4 KV blocks per query block; the rest are skipped.
+ *  - Budgets: the shared ranking of each query block's KV blocks is cut three times,
+ *    each cut rounded half up: c8 = floor((pct_fp8*N + 50)/100), c8m = floor(((pct_fp8 +
+ *    pct_mix)*N + 50)/100), ck = floor(((pct_fp8 + pct_mix + pct_fp4)*N + 50)/100). The top
+ *    n8 = c8 blocks are FP8, the next nm = c8m - c8 mixed (E4M3 Q K^T, E2M1 P V), the next
+ *    n4 = ck - c8m FP4; the rest are skipped.
  *  - Memory ownership: the caller allocates q, k, v, out and the workspace (device memory,
  *    size from da2_workspace_size); the library allocates no device memory and keeps no
  *    state (da2_forward_host creates and destroys three streams and a few events per call;
  *    da2_forward_noalloc uses a static device array of the library image).
  *  - Every call is asynchronous on `stream` (0 = legacy default stream) except the ones
  *    documented as synchronising. Argument errors are returned before anything is
- *    enqueued; a failed launch returns DA2_ERR_CUDA (see cudaGetLastError for detail).
+ *    enqueued; a failed CUDA call or launch returns DA2_ERR_CUDA, and da2_last_cuda_error
+ *    then gives its cudaError_t.
  *  - Supported: d in {64, 128}; any window with bs = ph*pw in {32, 64, 128}; N <= 4096;
- *    0 <= pct_fp8, pct_fp4 and pct_fp8 + pct_fp4 <= 100. Tensor pointers must be 16-byte
+ *    0 <= pct_fp8, pct_mix, pct_fp4 and pct_fp8 + pct_mix + pct_fp4 <= 100. Tensor pointers must be 16-byte
  *    aligned and the workspace 256-byte aligned (DA2_ERR_ALIGNMENT otherwise).
  */
 #ifndef DA2_H
@@ -63,6 +67,8 @@ typedef struct da2_config {
   int pct_fp8, pct_fp4; /* percent of KV blocks kept at FP8 / FP4; the rest is skipped */
   float sm_scale;       /* softmax scale; 0 selects 1/sqrt(d) */
   int flags;            /* DA2_FLAG_* bits */
+  int pct_mix;          /* percent of KV blocks in the mixed class (E4M3 scores, E2M1 P V),
+                           ranked between FP8 and FP4; 0 gives the two-class path */
 } da2_config;
 
 enum {
@@ -121,9 +127,10 @@ typedef enum da2_status {
      sv       fp32 [BH][d]   dequantisation scale of a V channel (channel amax / 448).
      vamax    fp32 [BH][d]   V channel amax (written by da2_prepare).
      qavg, qmax, kavg, kmax  fp32 [BH][N][d] pooled draft Q / K.
-     tags     u8 [BH][N][N]  0 skip, 1 FP4, 2 FP8 for (query block, KV block).
-     list8    i16 [BH][N][n8s], list4 i16 [BH][N][n4s]: kept KV blocks per query block
-              in ascending block order (n8s = max(n8,1), n4s = max(n4,1)).
+     tags     u8 [BH][N][N]  0 skip, 1 FP4, 2 FP8, 3 mixed for (query block, KV block).
+     list8    i16 [BH][N][n8s], list4 i16 [BH][N][n4s], listm i16 [BH][N][nms]: kept KV
+              blocks of each class per query block in ascending block order (n8s =
+              max(n8,1), n4s = max(n4,1), nms = max(nm,1)).
      scores   fp32 [BH][N][N] (only with DA2_FLAG_EXPORT_SCORES, else size 0).
      err      u32 device error word (0 = no error). */
 typedef struct da2_views {
@@ -132,6 +139,8 @@ typedef struct da2_views {
   size_t q8, k8, v8, q4, k4, v4, sfq4, sfk4, sfv4;
   size_t sq, sk, sv, vamax, qavg, qmax, kavg, kmax;
   size_t tags, list8, list4, scores, err, total;
+  int nm;               /* mixed KV blocks per query block */
+  size_t listm;
 } da2_views;
 
 /* Workspace bytes needed for `cfg` (host only, no CUDA call). */
@@ -207,6 +216,12 @@ da2_status da2_forward_noalloc(const da2_config* cfg, const void* q, const void*
    ignored). */
 da2_status da2_get_error(void* ws, size_t ws_bytes, const da2_config* cfg,
                          cudaStream_t stream, uint32_t* word);
+
+/* The cudaError_t of the calling host thread's most recent library call that returned
+   DA2_ERR_CUDA (cudaSuccess if none). The library checks every launch with
+   cudaGetLastError, which clears the runtime's own record, so this is where the code of,
+   say, cudaErrorLaunchOutOfResources is kept. Host only, no CUDA call. */
+int da2_last_cuda_error(void);
 
 /* Static string naming a status. */
 const char* da2_status_string(da2_status status);

@@ -38,7 +38,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned
 class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "d", "F", "Hf", "Wf", "ph", "pw",
                                              "pct_fp8", "pct_fp4")] + \
-               [("sm_scale", ctypes.c_float), ("flags", ctypes.c_int)]
+               [("sm_scale", ctypes.c_float), ("flags", ctypes.c_int), ("pct_mix", ctypes.c_int)]
 
 
 _VIEW_INTS = ("N", "bs", "T", "Tp", "ny", "nx", "n8", "n4", "kv4")
@@ -49,12 +49,16 @@ _VIEW_SIZES = ("tile8_qk", "tile4_qk", "tile8_v", "tile4_v", "sf_qk", "sf_v",
 
 
 class Views(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int) for n in _VIEW_INTS] + [(n, ctypes.c_size_t) for n in _VIEW_SIZES]
+    _fields_ = [(n, ctypes.c_int) for n in _VIEW_INTS] + [(n, ctypes.c_size_t) for n in _VIEW_SIZES] + \
+               [("nm", ctypes.c_int), ("listm", ctypes.c_size_t)]
 
 
 class DA2Error(RuntimeError):
     def __init__(self, fn, status):
-        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status})")
+        detail = ""
+        if status == 5 and _lib is not None and hasattr(_lib, "da2_last_cuda_error"):
+            detail = f", cudaError_t {_lib.da2_last_cuda_error()}"
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status}{detail})")
         self.status = status
 
 
@@ -84,6 +88,9 @@ def lib():
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
+        if hasattr(L, "da2_last_cuda_error"):
+            L.da2_last_cuda_error.argtypes = []
+            L.da2_last_cuda_error.restype = ctypes.c_int
         L.da2_status_string.argtypes = [ctypes.c_int]
         L.da2_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -92,13 +99,13 @@ def lib():
 
 EXPORTED = ("da2_workspace_size", "da2_workspace_views", "da2_prepare", "da2_draft_select",
             "da2_attention", "da2_forward", "da2_forward_host", "da2_get_error",
-            "da2_status_string", "da2_forward_noalloc")
+            "da2_status_string", "da2_forward_noalloc", "da2_last_cuda_error")
 
 
 def config(w, flags: int = 0, sm_scale: float = 0.0) -> Config:
     """da2_config of a synth.Workload (or any object with the same fields)."""
     return Config(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, w.pct_fp8, w.pct_fp4,
-                  float(sm_scale), int(flags))
+                  float(sm_scale), int(flags), int(getattr(w, "pct_mix", 0)))
 
 
 def _check(fn, st):
@@ -125,7 +132,7 @@ def workspace_size(cfg: Config) -> int:
 def workspace_views(cfg: Config) -> dict:
     v = Views()
     _check("da2_workspace_views", lib().da2_workspace_views(ctypes.byref(cfg), ctypes.byref(v)))
-    return {n: getattr(v, n) for n in _VIEW_INTS + _VIEW_SIZES}
+    return {n: getattr(v, n) for n in _VIEW_INTS + _VIEW_SIZES + ("nm", "listm")}
 
 
 def prepare(cfg, q, k, v, ws, stream=None):

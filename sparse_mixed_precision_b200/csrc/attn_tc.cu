@@ -6,9 +6,11 @@
 // Diffusion via Low-Resolution Attention Guidance", Abstract: the output is restored to
 // the original token order after the block-sparse attention.
 //
-// Per work item (b, h, query block i): the FP8 phase visits list8[i], then the FP4 phase
-// visits list4[i], both in ascending block order, with ONE running row max m, ONE running
-// sum l and ONE fp32 accumulator O in tensor memory. For each visited block j:
+// Per work item (b, h, query block i): the FP8 phase visits list8[i], the mixed phase
+// listm[i] (E4M3 scores, E2M1 P V), then the FP4 phase list4[i], each in ascending block
+// order, with ONE running row max m, ONE running sum l and ONE fp32 accumulator O in tensor
+// memory. For each visited block j (S at the block's score precision, P V at its P V
+// precision):
 //   S = Q' K_j'^T            tcgen05.mma kind::f8f6f4 (E4M3) or kind::mxf4nvf4 (E2M1 with
 //                            E4M3 scales per 16 along d), fp32 in TMEM
 //   m_new = max(m, rowmax(S * s_q s_k sm_scale)), padded keys masked
@@ -347,7 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
   Bars* bars = reinterpret_cast<Bars*>(sm + kBar);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = g.N, BH = g.B * g.H;
-  const int n8 = g.n8, nb = g.n8 + g.n4;
+  // phases: blocks t < n8 FP8, n8 <= t < n8m mixed (E4M3 scores, E2M1 P V), then FP4
+  const int n8 = g.n8, n8m = g.n8 + g.nm, nb = g.n8 + g.nm + g.n4;
   const int total = BH * N;
   constexpr int KV4 = BS < 64 ? 64 : BS;
   // work items of this CTA: blockIdx.x + m gridDim.x; round k takes m = 2k (A), 2k+1 (B)
@@ -413,19 +416,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
     // ===================== producer =====================
     if (lane == 0 && nb > 0) {
       uint32_t gkv = 0;
-      auto list_j = [&](const int16_t* l8, const int16_t* l4, int t) {
-        const int j = t < n8 ? l8[t] : l4[t - n8];
+      auto list_j = [&](const int16_t* l8, const int16_t* lm, const int16_t* l4, int t) {
+        const int j = t < n8 ? l8[t] : (t < n8m ? lm[t - n8] : l4[t - n8m]);
         return (j < 0 || j >= N) ? 0 : j;
       };
-      auto kv_prefetch = [&](int bh, int j, bool fp8) {
+      // K at 8 bits for FP8 and mixed blocks, V at 8 bits for FP8 blocks only
+      auto kv_prefetch = [&](int bh, int j, int t) {
         const size_t kj = (size_t)bh * N + j;
-        if (fp8) {
-          tc::prefetch_l2(w.k8 + kj * w.tile8_qk, BS * D);
-          tc::prefetch_l2(w.v8 + kj * w.tile8_v, BS * D);
-        } else {
-          tc::prefetch_l2(w.k4 + kj * w.tile4_qk, BS * D / 2);
-          tc::prefetch_l2(w.v4 + kj * w.tile4_v, D * KV4 / 2);
-        }
+        if (t < n8m) tc::prefetch_l2(w.k8 + kj * w.tile8_qk, BS * D);
+        else tc::prefetch_l2(w.k4 + kj * w.tile4_qk, BS * D / 2);
+        if (t < n8) tc::prefetch_l2(w.v8 + kj * w.tile8_v, BS * D);
+        else tc::prefetch_l2(w.v4 + kj * w.tile4_v, D * KV4 / 2);
       };
       bool dead = false;                // a wait ran out: issue nothing more
       int q_rounds[2] = {0, 0};         // Q tiles loaded per tile
@@ -434,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         const int nx = has_tile(k, 1) ? 2 : 1;
         int bhx[2], ix[2];
         const int16_t* l8x[2];
+        const int16_t* lmx[2];
         const int16_t* l4x[2];
         for (int x = 0; x < nx && !dead; ++x) {
           const int item = item_of(k, x);
@@ -441,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           ix[x] = item - bhx[x] * N;
           const size_t qi = (size_t)bhx[x] * N + ix[x];
           l8x[x] = w.list8 + qi * w.n8s;
+          lmx[x] = w.listm + qi * w.nms;
           l4x[x] = w.list4 + qi * w.n4s;
           TileBars* tb = &bars->tb[x];
           if (!wait_bar(&tb->q_empty, (k & 1) ^ 1, w.err, g.wait_ns)) { dead = true; break; }
@@ -454,13 +457,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         }
         if (dead) break;
         for (int t = 0; t < kPrefetch / 2 && t < nb; ++t)
-          for (int x = 0; x < nx; ++x) kv_prefetch(bhx[x], list_j(l8x[x], l4x[x], t), t < n8);
+          for (int x = 0; x < nx; ++x) kv_prefetch(bhx[x], list_j(l8x[x], lmx[x], l4x[x], t), t);
         for (int t = 0; t < nb && !dead; ++t) {
-          const bool fp8 = t < n8;
+          const bool k8 = t < n8m, v8 = t < n8;
           for (int x = 0; x < nx; ++x) {
             if (t + kPrefetch / 2 < nb)
-              kv_prefetch(bhx[x], list_j(l8x[x], l4x[x], t + kPrefetch / 2), t + kPrefetch / 2 < n8);
-            const int j = list_j(l8x[x], l4x[x], t);
+              kv_prefetch(bhx[x], list_j(l8x[x], lmx[x], l4x[x], t + kPrefetch / 2), t + kPrefetch / 2);
+            const int j = list_j(l8x[x], lmx[x], l4x[x], t);
             const size_t kj = (size_t)bhx[x] * N + j;
             const uint32_t s = gkv % kStages, ks = gkv / kStages;
             if (stall && gkv == 0) {      // withhold the first K/V tile: its consumer's wait runs out
@@ -469,16 +472,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
             }
             if (!wait_bar(&bars->kv_empty[s], (ks & 1) ^ 1, w.err, g.wait_ns)) { dead = true; break; }
             uint8_t* st = sm + kStage0 + s * kStageBytes;
-            if (fp8) {
-              tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * BS * D);
+            const uint32_t kbytes = k8 ? BS * D : BS * D / 2 + (uint32_t)w.sf_qk;
+            const uint32_t vbytes = v8 ? BS * D : D * KV4 / 2 + (uint32_t)w.sf_v;
+            tc::mbar_arrive_expect_tx(&bars->kv_full[s], kbytes + vbytes);
+            if (k8) {
               tc::bulk_g2s(st + kStK, w.k8 + kj * w.tile8_qk, BS * D, &bars->kv_full[s]);
+            } else {
+              tc::bulk_g2s(st + kStK, w.k4 + kj * w.tile4_qk, BS * D / 2, &bars->kv_full[s]);
+              tc::bulk_g2s(st + kStSFK, w.sfk4 + kj * w.sf_qk, (uint32_t)w.sf_qk, &bars->kv_full[s]);
+            }
+            if (v8) {
               tc::bulk_g2s(st + kStV, w.v8 + kj * w.tile8_v, BS * D, &bars->kv_full[s]);
             } else {
-              const uint32_t bytes = BS * D / 2 + D * KV4 / 2 + (uint32_t)w.sf_qk + (uint32_t)w.sf_v;
-              tc::mbar_arrive_expect_tx(&bars->kv_full[s], bytes);
-              tc::bulk_g2s(st + kStK, w.k4 + kj * w.tile4_qk, BS * D / 2, &bars->kv_full[s]);
               tc::bulk_g2s(st + kStV, w.v4 + kj * w.tile4_v, D * KV4 / 2, &bars->kv_full[s]);
-              tc::bulk_g2s(st + kStSFK, w.sfk4 + kj * w.sf_qk, (uint32_t)w.sf_qk, &bars->kv_full[s]);
               tc::bulk_g2s(st + kStSFV, w.sfv4 + kj * w.sf_v, (uint32_t)w.sf_v, &bars->kv_full[s]);
             }
             ++gkv;
@@ -512,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         const uint32_t kvbase = 2u * gbase;                  // K/V stages of earlier rounds (2 tiles each)
         dead = !wait_bar(&tb->q_full, k & 1, w.err, g.wait_ns);
         tc::fence_after_sync();
-        if (!dead && nb > n8)
+        if (!dead && nb > n8m)                               // blocks with E2M1 scores follow
           for (int kb = 0; kb < D / 64; ++kb)
             tc::cp_sf_atom(tmem + kColSFQ + 8 * x + kb * 4, qs + kSFQ + kb * 512);
         // The S region is taken in the order A0 B0 A1 B1 ... (A0 A1 ... when B is absent),
@@ -531,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           if (!wait_bar(&bars->kv_full[s], (seq / kStages) & 1, w.err, g.wait_ns)) return false;
           tc::fence_after_sync();
           const uint8_t* st = sm + kStage0 + s * kStageBytes;
-          if (t < n8) {
+          if (t < n8m) {                                      // FP8 and mixed blocks: E4M3 scores
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)
               tc::mma_e4m3(tmem + kColS, tc::sdesc(qs + kQ8 + kk * 256, 128, D * 8),
@@ -623,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       }
       const float sq = w.sq[qi];
       const int16_t* l8 = w.list8 + qi * w.n8s;
+      const int16_t* lm = w.listm + qi * w.nms;
       const int16_t* l4 = w.list4 + qi * w.n4s;
       float m = -INFINITY, l = 0.0f;
       // Block index j and key scale s_k[j] of every visited block, fetched 32 blocks at a
@@ -632,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       const float cq = sq * g.sm_scale * kLog2e;
       const float* skh = w.sk + (size_t)bh * N;
       auto list_j = [&](int t) -> int {
-        const int j = t < nb ? (t < n8 ? l8[t] : l4[t - n8]) : 0;
+        const int j = t < nb ? (t < n8 ? l8[t] : (t < n8m ? lm[t - n8] : l4[t - n8m])) : 0;
         return (j < 0 || j >= N) ? 0 : j;
       };
       int jA = list_j(lane), jB = list_j(32 + lane), jC = list_j(64 + lane);

@@ -15,6 +15,7 @@ constexpr float kE4M3Max = 448.0f;
 struct Geo {
   int B, H, d, F, Hf, Wf, ph, pw;
   int ny, nx, N, bs, T, Tp, n8, n4, kv4;
+  int nm;     // mixed KV blocks per query block (E4M3 scores, E2M1 P V)
   float sm_scale;
   int flags;
   int bthd;   // q, k, v, out token-major [B,T,H,d] instead of [B,H,T,d]
@@ -37,10 +38,10 @@ struct Ws {
   uint8_t *q8, *k8, *v8, *q4, *k4, *v4, *sfq4, *sfk4, *sfv4;
   float *sq, *sk, *sv, *vamax, *qavg, *qmax, *kavg, *kmax, *scores;
   uint8_t* tags;
-  int16_t *list8, *list4;
+  int16_t *list8, *list4, *listm;
   uint32_t* err;
   size_t tile8_qk, tile4_qk, tile8_v, tile4_v, sf_qk, sf_v;
-  int n8s, n4s;
+  int n8s, n4s, nms;
 };
 
 // Device error word bits.

@@ -26,7 +26,8 @@ da2_status check_config(const da2_config* c) {
   if (!c) return DA2_ERR_INVALID_ARG;
   if (c->B <= 0 || c->H <= 0 || c->F <= 0 || c->Hf <= 0 || c->Wf <= 0 || c->ph <= 0 || c->pw <= 0)
     return DA2_ERR_INVALID_ARG;
-  if (c->pct_fp8 < 0 || c->pct_fp4 < 0 || c->pct_fp8 + c->pct_fp4 > 100) return DA2_ERR_INVALID_ARG;
+  if (c->pct_fp8 < 0 || c->pct_fp4 < 0 || c->pct_mix < 0 || c->pct_fp8 + c->pct_mix + c->pct_fp4 > 100)
+    return DA2_ERR_INVALID_ARG;
   if (!(c->sm_scale >= 0.0f) || std::isinf(c->sm_scale)) return DA2_ERR_INVALID_ARG;
   if (c->flags & ~(DA2_FLAG_EXPORT_SCORES | DA2_FLAG_NO_MASS_CORRECTION | DA2_FLAG_LAYOUT_BTHD |
                    DA2_FLAG_TEST_STALL))
@@ -49,8 +50,12 @@ void fill_views(const da2_config* c, da2_views* v) {
   v->bs = c->ph * c->pw;
   v->T = c->F * c->Hf * c->Wf;
   v->Tp = v->N * v->bs;
-  v->n8 = (c->pct_fp8 * v->N + 50) / 100;
-  v->n4 = ((c->pct_fp8 + c->pct_fp4) * v->N + 50) / 100 - v->n8;
+  const int c8 = (c->pct_fp8 * v->N + 50) / 100;
+  const int c8m = ((c->pct_fp8 + c->pct_mix) * v->N + 50) / 100;
+  const int ck = ((c->pct_fp8 + c->pct_mix + c->pct_fp4) * v->N + 50) / 100;
+  v->n8 = c8;
+  v->nm = c8m - c8;
+  v->n4 = ck - c8m;
   v->kv4 = v->bs < 64 ? 64 : v->bs;
   const size_t d = c->d, bs = v->bs, N = v->N, BH = (size_t)c->B * c->H;
   v->tile8_qk = bs * d;
@@ -59,7 +64,7 @@ void fill_views(const da2_config* c, da2_views* v) {
   v->tile4_v = d * v->kv4 / 2;
   v->sf_qk = (d / 64) * 512;
   v->sf_v = (v->kv4 / 64) * 512;
-  const size_t n8s = v->n8 > 0 ? v->n8 : 1, n4s = v->n4 > 0 ? v->n4 : 1;
+  const size_t n8s = v->n8 > 0 ? v->n8 : 1, n4s = v->n4 > 0 ? v->n4 : 1, nms = v->nm > 0 ? v->nm : 1;
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + bytes); return o; };
   v->q8 = take(BH * N * v->tile8_qk);
@@ -82,6 +87,7 @@ void fill_views(const da2_config* c, da2_views* v) {
   v->tags = take(BH * N * N);
   v->list8 = take(BH * N * n8s * 2);
   v->list4 = take(BH * N * n4s * 2);
+  v->listm = take(BH * N * nms * 2);
   v->scores = take((c->flags & DA2_FLAG_EXPORT_SCORES) ? BH * N * N * 4 : 0);
   v->err = take(4);
   v->total = off;
@@ -91,7 +97,7 @@ Geo make_geo(const da2_config* c, const da2_views& v) {
   Geo g;
   g.B = c->B; g.H = c->H; g.d = c->d; g.F = c->F; g.Hf = c->Hf; g.Wf = c->Wf;
   g.ph = c->ph; g.pw = c->pw; g.ny = v.ny; g.nx = v.nx; g.N = v.N; g.bs = v.bs;
-  g.T = v.T; g.Tp = v.Tp; g.n8 = v.n8; g.n4 = v.n4; g.kv4 = v.kv4;
+  g.T = v.T; g.Tp = v.Tp; g.n8 = v.n8; g.n4 = v.n4; g.kv4 = v.kv4; g.nm = v.nm;
   g.sm_scale = c->sm_scale > 0.0f ? c->sm_scale : 1.0f / std::sqrt((float)c->d);
   g.flags = c->flags;
   g.bthd = (c->flags & DA2_FLAG_LAYOUT_BTHD) ? 1 : 0;
@@ -118,11 +124,13 @@ Ws make_ws(void* base, const da2_views& v) {
   w.tags = b + v.tags;
   w.list8 = reinterpret_cast<int16_t*>(b + v.list8);
   w.list4 = reinterpret_cast<int16_t*>(b + v.list4);
+  w.listm = reinterpret_cast<int16_t*>(b + v.listm);
   w.err = reinterpret_cast<uint32_t*>(b + v.err);
   w.tile8_qk = v.tile8_qk; w.tile4_qk = v.tile4_qk; w.tile8_v = v.tile8_v; w.tile4_v = v.tile4_v;
   w.sf_qk = v.sf_qk; w.sf_v = v.sf_v;
   w.n8s = v.n8 > 0 ? v.n8 : 1;
   w.n4s = v.n4 > 0 ? v.n4 : 1;
+  w.nms = v.nm > 0 ? v.nm : 1;
   return w;
 }
 
@@ -139,7 +147,15 @@ da2_status setup(const da2_config* cfg, void* ws, size_t ws_bytes, da2_views* v,
   return DA2_OK;
 }
 
-da2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DA2_OK : DA2_ERR_CUDA; }
+// CUDA error of the calling thread's last failed library call (the launch's own
+// cudaGetLastError has consumed it by the time the caller could ask the runtime).
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+da2_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return DA2_OK;
+  g_last_cuda = e;
+  return DA2_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -208,7 +224,7 @@ da2_status forward_host_serial(const da2_config* cfg, const void* q_host, const 
   cudaError_t e = cudaMemcpyAsync(dq, q_host, bytes, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, bytes, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, bytes, cudaMemcpyHostToDevice, stream);
-  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   const da2_status s = da2_forward(cfg, dq, dk, dv, dout, ws, ws_bytes, stream);
   if (s != DA2_OK) return s;
   e = cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, stream);
@@ -347,10 +363,12 @@ da2_status da2_get_error(void* ws, size_t ws_bytes, const da2_config* cfg, cudaS
   cudaError_t e = cudaMemcpyAsync(&h, w.err, 4, cudaMemcpyDeviceToHost, stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(w.err, 0, 4, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   *word = h;
   return h ? DA2_ERR_TIMEOUT : DA2_OK;
 }
+
+int da2_last_cuda_error(void) { return (int)g_last_cuda; }
 
 const char* da2_status_string(da2_status s) {
   switch (s) {

@@ -11,7 +11,8 @@
 // One CTA takes R query blocks of one (b, h): it forms both draft logit rows against all N
 // key blocks (fp32 FMA), turns each into a row softmax, averages the two maps into the
 // score, and each warp ranks its rows with an exact radix select over the score bits
-// (ties broken by the lower block index), then writes tags and the ascending index lists.
+// (ties broken by the lower block index), then writes tags and the ascending index lists of
+// the kept classes (FP8, mixed, FP4).
 #include "common.cuh"
 
 namespace da2 {
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kDraftThreads) k_draft_select(Geo g, Ws w, int
   }
   __syncthreads();
 
-  const int nk = g.n8 + g.n4;
+  const int n8m = g.n8 + g.nm, nk = g.n8 + g.nm + g.n4;   // the ranking's cuts
   uint32_t* h = hist + warp * 256;
   for (int r = warp; r < rows; r += kDraftWarps) {
     float* ra = la + r * N;
@@ -165,35 +166,46 @@ __global__ void __launch_bounds__(kDraftThreads) k_draft_select(Geo g, Ws w, int
     }
     __syncwarp();
     const uint32_t* keys = reinterpret_cast<const uint32_t*>(ra);
-    uint32_t T8 = 0xFFFFFFFFu, Tk = 0xFFFFFFFFu;
-    int need8 = 0, needk = 0;
+    // the three cuts of the ranking: n8-th, (n8 + nm)-th and nk-th largest score
+    uint32_t T8 = 0xFFFFFFFFu, Tm = 0xFFFFFFFFu, Tk = 0xFFFFFFFFu;
+    int need8 = 0, needm = 0, needk = 0;
     if (g.n8 > 0) warp_radix_select(keys, N, g.n8, h, T8, need8);
+    if (g.nm > 0) warp_radix_select(keys, N, n8m, h, Tm, needm);
     if (nk > 0) warp_radix_select(keys, N, nk, h, Tk, needk);
-    int eq8 = 0, eqk = 0, c8 = 0, c4 = 0;
+    int eq8 = 0, eqm = 0, eqk = 0, c8 = 0, cm = 0, c4 = 0;
     uint8_t* trow = w.tags + row * N;
     int16_t* l8 = w.list8 + row * w.n8s;
+    int16_t* lmx = w.listm + row * w.nms;
     int16_t* l4 = w.list4 + row * w.n4s;
     const uint32_t lt = (1u << lane) - 1u;
     for (int j0 = 0; j0 < N; j0 += 32) {
       const int j = j0 + lane;
       const bool ok = j < N;
       const uint32_t key = ok ? keys[j] : 0u;
+      // keys equal to a cut value belong above it in block order, as many as the cut needs
       const uint32_t e8 = __ballot_sync(0xffffffffu, ok && g.n8 > 0 && key == T8);
+      const uint32_t em = __ballot_sync(0xffffffffu, ok && g.nm > 0 && key == Tm);
       const uint32_t ek = __ballot_sync(0xffffffffu, ok && nk > 0 && key == Tk);
       const bool in8 = ok && g.n8 > 0 && (key > T8 || (key == T8 && eq8 + __popc(e8 & lt) < need8));
+      const bool in8m = in8 || (ok && g.nm > 0 && (key > Tm || (key == Tm && eqm + __popc(em & lt) < needm)));
       const bool ink = ok && nk > 0 && (key > Tk || (key == Tk && eqk + __popc(ek & lt) < needk));
       eq8 += __popc(e8);
+      eqm += __popc(em);
       eqk += __popc(ek);
-      const bool in4 = ink && !in8;
-      const uint32_t b8 = __ballot_sync(0xffffffffu, in8), b4 = __ballot_sync(0xffffffffu, in4);
-      const int p8 = c8 + __popc(b8 & lt), p4 = c4 + __popc(b4 & lt);
+      const bool inm = in8m && !in8;
+      const bool in4 = ink && !in8m;
+      const uint32_t b8 = __ballot_sync(0xffffffffu, in8), bm = __ballot_sync(0xffffffffu, inm),
+                     b4 = __ballot_sync(0xffffffffu, in4);
+      const int p8 = c8 + __popc(b8 & lt), pm = cm + __popc(bm & lt), p4 = c4 + __popc(b4 & lt);
       if (in8 && p8 < g.n8) l8[p8] = (int16_t)j;
+      if (inm && pm < g.nm) lmx[pm] = (int16_t)j;
       if (in4 && p4 < g.n4) l4[p4] = (int16_t)j;
       c8 += __popc(b8);
+      cm += __popc(bm);
       c4 += __popc(b4);
-      if (ok) trow[j] = in8 ? 2 : (in4 ? 1 : 0);
+      if (ok) trow[j] = in8 ? 2 : (inm ? 3 : (in4 ? 1 : 0));
     }
-    if (lane == 0 && (c8 != g.n8 || c4 != g.n4)) set_error(w.err, kErrBadIndex);
+    if (lane == 0 && (c8 != g.n8 || cm != g.nm || c4 != g.n4)) set_error(w.err, kErrBadIndex);
   }
 }
 

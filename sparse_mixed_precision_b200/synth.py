@@ -58,6 +58,8 @@ WORKLOADS = {
     "wan720": Workload("wan720", 1, 40, 128, 21, 45, 80, 8, 16, 10, 30, 4, False, 1002),
     "hunyuan720": Workload("hunyuan720", 1, 24, 128, 33, 45, 80, 8, 16, 5, 25, 0, True, 1003),
 }
+# The 720p layer with the mixed class between FP8 and FP4 (FP8 10 / mixed 10 / FP4 20 / skip 60).
+WORKLOADS["wan720mix"] = Workload("wan720mix", 1, 40, 128, 21, 45, 80, 8, 16, 10, 20, 4, False, 1002, 10)
 SWEEP_BUDGETS = [(100, 0), (0, 100), (25, 0), (10, 30), (5, 45)]
 for _i, (_p8, _p4) in enumerate(SWEEP_BUDGETS):
     WORKLOADS[f"sweep{_i}"] = Workload(f"sweep{_i}", 2, 40, 128, 21, 45, 80, 8, 16,

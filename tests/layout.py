@@ -95,6 +95,12 @@ class WsReader:
         l4 = self._bytes("list4", bh0, bh1, v["N"] * n4s * 2).view(np.int16).reshape(bh1 - bh0, v["N"], n4s)
         return l8[..., : v["n8"]].astype(np.int64), l4[..., : v["n4"]].astype(np.int64)
 
+    def listm(self, bh0, bh1):
+        v = self.v
+        nms = max(v["nm"], 1)
+        lm = self._bytes("listm", bh0, bh1, v["N"] * nms * 2).view(np.int16).reshape(bh1 - bh0, v["N"], nms)
+        return lm[..., : v["nm"]].astype(np.int64)
+
     def scores(self, bh0, bh1):
         N = self.v["N"]
         return self.f32("scores", bh0, bh1, N * N).reshape(bh1 - bh0, N, N)

@@ -41,7 +41,8 @@ def test_workspace_views_consistent():
         g = O.geometry(w)
         assert (v["N"], v["bs"], v["T"], v["Tp"], v["n8"], v["n4"]) == (g.N, g.bs, g.T, g.Tp, g.n8, g.n4)
         offs = sorted((v[k], k) for k in ("q8", "k8", "v8", "q4", "k4", "v4", "sfq4", "sfk4",
-                                           "sfv4", "sq", "sk", "sv", "tags", "list8", "err"))
+                                           "sfv4", "sq", "sk", "sv", "tags", "list8", "list4",
+                                           "listm", "err"))
         assert all(o % 256 == 0 for o, _ in offs)
         assert len({o for o, _ in offs}) == len(offs)
     # exporting scores grows the workspace by 4 B H N^2 (rounded to 256)
@@ -123,3 +124,23 @@ def test_noalloc_host_side_refusals():
     # reading the scratch's error word needs a valid configuration first
     word = ctypes.c_uint32()
     assert L.da2_get_error(None, 0, ctypes.byref(bad), None, ctypes.byref(word)) == 1
+
+
+def test_last_cuda_error_is_host_only():
+    # no library call has failed with DA2_ERR_CUDA in this thread: cudaSuccess
+    assert da2.lib().da2_last_cuda_error() == 0
+
+
+def test_mixed_budget_counts_and_limits():
+    # three cumulative cuts, each rounded half up; the percentages may not exceed 100
+    L = da2.lib()
+    n = ctypes.c_size_t()
+    w = scaled(WORKLOADS["wan720"], pct_fp8=10, pct_mix=10, pct_fp4=20)
+    v = da2.workspace_views(da2.config(w))
+    assert (v["n8"], v["nm"], v["n4"]) == (63, 63, 126)
+    v0 = da2.workspace_views(da2.config(WORKLOADS["wan720"]))
+    assert (v0["n8"], v0["nm"], v0["n4"]) == (63, 0, 189)
+    bad = da2.config(scaled(WORKLOADS["tiny"], pct_fp8=40, pct_mix=40, pct_fp4=30))
+    assert L.da2_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == 1
+    neg = da2.config(scaled(WORKLOADS["tiny"], pct_mix=-1))
+    assert L.da2_workspace_size(ctypes.byref(neg), ctypes.byref(n)) == 1

@@ -70,14 +70,18 @@ def check_selection(views, rd, bh, P, g):
     l8, l4 = rd.lists(bh, bh + 1)
     # the CUDA path's own fp32 scores, ranked by the oracle, give exactly its tags and lists
     sc = rd.scores(bh, bh + 1)[0].astype(np.float64)
-    t2, a8, a4 = O.rank(sc, g.n8, g.n4)
-    assert np.array_equal(t2, tags) and np.array_equal(a8, l8[0]) and np.array_equal(a4, l4[0])
+    r2 = O.rank_classes(sc, g.n8, g.nm, g.n4)
+    assert np.array_equal(r2["tags"], tags) and np.array_equal(r2["list8"], l8[0])
+    assert np.array_equal(r2["list4"], l4[0])
+    if g.nm > 0:
+        assert np.array_equal(r2["listm"], rd.listm(bh, bh + 1)[0])
     # against the oracle's fp64 scores: mismatches only at near-ties across a cut
     ref = sel["scores"][0, 0]
     excused = 0
+    c8m, ck = g.n8 + g.nm, g.n8 + g.nm + g.n4
     for r in np.flatnonzero((tags != sel["tags"][0, 0]).any(axis=1)):
         order = np.lexsort((np.arange(g.N), -ref[r]))
-        cuts = [ref[r, order[c]] for c in (g.n8 - 1, g.n8, g.n8 + g.n4 - 1, g.n8 + g.n4)
+        cuts = [ref[r, order[c]] for c in (g.n8 - 1, g.n8, c8m - 1, c8m, ck - 1, ck)
                 if 0 <= c < g.N]
         tol = TIE_REL * ref[r].max()
         for j in np.flatnonzero(tags[r] != sel["tags"][0, 0, r]):
@@ -86,10 +90,11 @@ def check_selection(views, rd, bh, P, g):
     return l8, l4, excused
 
 
-def check_attention(w, views, P, l8, l4, out_bh, blocks, g):
+def check_attention(w, views, P, l8, l4, out_bh, blocks, g, lm=None):
     ops = O.operands_quantised(P["Q"], P["K"], P["V"])
     ob = O.attention(ops, P["valid"], l8[None, None], l4[None, None], g.sm_scale, True,
-                     blocks=[(0, 0, i) for i in blocks])
+                     blocks=[(0, 0, i) for i in blocks],
+                     listm=None if lm is None else lm[None, None])
     blk, slot = O.token_block_slot(g)
     sel = np.isin(blk, blocks)
     ref = ob[0, 0][blk[sel], slot[sel]]
@@ -296,4 +301,32 @@ def test_small_shapes_full_parity(kw):
         l8, l4, _ = check_selection(views, rd, h, P, g)
         check_attention(w, views, P, l8[0], l4[0], out[0, h].float().cpu().numpy(),
                         list(range(g.N)), g)
+    assert torch.isfinite(out).all()
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", dict(pct_fp8=10, pct_mix=15, pct_fp4=25)),
+    ("tiny", dict(pct_fp8=0, pct_mix=100, pct_fp4=0)),
+    ("wan720", dict(H=3, F=3, pct_fp8=10, pct_mix=10, pct_fp4=20)),
+    ("wan480", dict(H=2, F=3, pct_fp8=5, pct_mix=20, pct_fp4=15)),
+], ids=["tiny-3class", "tiny-all-mixed", "wan720-3class", "wan480-3class"])
+def test_mixed_class_parity(name, kw):
+    # the mixed class (E4M3 scores, E2M1 P V) between FP8 and FP4: tags and all three lists
+    # exactly as the oracle ranks the CUDA scores, outputs within the tolerance
+    w = scaled(WORKLOADS[name], **kw)
+    q, k, v = generate(w, device="cuda")
+    cfg, views, ws, out = run_cuda(w, q, k, v)
+    rd = WsReader(ws, views, w.d)
+    g = O.geometry(scaled(w, B=1, H=1))
+    assert views["nm"] == g.nm and g.nm > 0
+    for h in range(w.H):
+        qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+        P = check_prep(w, views, rd, h, qh, kh, vh)
+        l8, l4, _ = check_selection(views, rd, h, P, g)
+        lm = rd.listm(h, h + 1)
+        tags = rd.tags(h, h + 1)[0]
+        assert ((tags == 3).sum(axis=1) == g.nm).all()
+        blocks = list(range(g.N)) if g.N <= 64 else sorted(set(
+            [0, g.N - 1] + list(np.random.default_rng(h).choice(g.N, 6, replace=False))))
+        check_attention(w, views, P, l8[0], l4[0], out[0, h].float().cpu().numpy(), blocks, g, lm=lm[0])
     assert torch.isfinite(out).all()
