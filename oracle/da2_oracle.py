@@ -60,6 +60,8 @@ class Geometry:
     n4: int       # FP4 blocks per query block
     sm_scale: float
     nm: int = 0   # mixed blocks per query block (E4M3 scores, E2M1 P V)
+    n4max: int = 0  # FP4 list length with the adaptive budget (n4 when it is off)
+    tau: float = 0.0  # adaptive budget threshold on the draft score (0: off)
 
 
 def budget_counts(N: int, pct_fp8: int, pct_fp4: int) -> tuple[int, int]:
@@ -93,10 +95,13 @@ def geometry(w) -> Geometry:
     ny, nx = -(-w.Hf // w.ph), -(-w.Wf // w.pw)
     N = w.F * ny * nx
     bs = w.ph * w.pw
-    n8, nm, n4 = budget_counts3(N, w.pct_fp8, getattr(w, "pct_mix", 0), w.pct_fp4)
+    pm = getattr(w, "pct_mix", 0)
+    n8, nm, n4 = budget_counts3(N, w.pct_fp8, pm, w.pct_fp4)
+    tau = float(getattr(w, "adapt_tau", 0.0))
+    n4max = budget_counts3(N, w.pct_fp8, pm, w.pct_fp4_max)[2] if tau > 0 else n4
     sm = getattr(w, "sm_scale", 0.0) or 1.0 / math.sqrt(w.d)
     return Geometry(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, ny, nx, N, bs,
-                    w.F * w.Hf * w.Wf, N * bs, n8, n4, sm, nm)
+                    w.F * w.Hf * w.Wf, N * bs, n8, n4, sm, nm, n4max, tau)
 
 
 def token_block_slot(g: Geometry):
@@ -372,6 +377,44 @@ def rank_classes(scores, n8: int, nm: int, n4: int):
                 list4=lists[TAG_FP4].reshape(lead + (n4,)))
 
 
+def rank_adaptive(scores, n8: int, nm: int, n4: int, n4max: int, tau: float):
+    """The shared ranking with an error-bound-driven FP4 budget per row.
+
+    [DA2] Abstract: the analysis separates the sparsification error from the
+    attention-weighted quantisation error and establishes when recovering skipped
+    interactions with low-bit computation tightens the output-error bound. Reading: a
+    skipped block j adds about its attention mass w_j times the output's deviation to the
+    sparsification term; kept at FP4 it adds w_j times FP4's much smaller relative error to
+    the quantisation term, so recovering it tightens the bound by an amount proportional to
+    w_j. Per row the blocks ranked after the fixed budgets therefore join the FP4 class, in
+    rank order, while their draft score (the estimated block mass) is at least tau, until
+    the row holds n4max FP4 blocks. list4 keeps ascending block order and is padded to n4max
+    entries with -1 (no block); count4 holds each row's FP4 count.
+    """
+    r = rank_classes(scores, n8, nm, n4)
+    sc = np.asarray(scores)
+    lead = sc.shape[:-1]
+    N = sc.shape[-1]
+    flat = sc.reshape(-1, N)
+    tags = r["tags"].reshape(-1, N).copy()
+    l4 = np.full((flat.shape[0], n4max), -1, dtype=np.int64)
+    cnt = np.zeros(flat.shape[0], dtype=np.int64)
+    j = np.arange(N)
+    ck, ckmax = n8 + nm + n4, min(n8 + nm + n4max, N)
+    base4 = r["list4"].reshape(-1, n4)
+    for row in range(flat.shape[0]):
+        order = np.lexsort((j, -flat[row]))
+        extra = [b for b in order[ck:ckmax] if flat[row, b] >= tau]
+        # the candidates are in descending score order: the recovered ones form a prefix
+        assert extra == list(order[ck:ck + len(extra)])
+        tags[row, extra] = TAG_FP4
+        kept = np.sort(np.concatenate([base4[row], np.array(extra, dtype=np.int64)]))
+        l4[row, :len(kept)] = kept
+        cnt[row] = len(kept)
+    return dict(tags=tags.reshape(lead + (N,)), list8=r["list8"], listm=r["listm"],
+                list4=l4.reshape(lead + (n4max,)), count4=cnt.reshape(lead))
+
+
 def rank(scores, n8: int, n4: int):
     """The two-class ranking (no mixed blocks): tags, list8 and list4 of `rank_classes`."""
     r = rank_classes(scores, n8, 0, n4)
@@ -454,6 +497,8 @@ def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
                 for prec, pprec, lst in phases:       # score precision, P V precision
                     qi = ops.q[prec][b, h, i]
                     for j in lst:
+                        if j < 0:                     # padding of an adaptive FP4 list
+                            continue
                         S = sm_scale * (qi @ ops.k[prec][b, h, j].T)
                         S[:, ~valid[j]] = -np.inf
                         m_new = np.maximum(m, S.max(axis=1))
@@ -509,7 +554,8 @@ def error_decomposition(q, k, v, valid, list8, list4, ops_q: Operands, sm_scale,
         for h in range(H):
             for i in range(N):
                 kept[b, h, i, list8[b, h, i]] = True
-                kept[b, h, i, list4[b, h, i]] = True
+                l4 = list4[b, h, i]
+                kept[b, h, i, l4[l4 >= 0]] = True          # -1 pads an adaptive FP4 list
     all8 = np.broadcast_to(np.arange(N), (B, H, N, N))
     none = np.zeros((B, H, N, 0), dtype=np.int64)
     O = attention(ops_x, valid, all8, none, sm_scale, quantise_p=False)
@@ -577,7 +623,10 @@ def draft_select(prep, mass_correction=True):
     g = prep["g"]
     sc = draft_scores(prep["qavg"], prep["kavg"], prep["qmax"], prep["kmax"],
                       prep["counts"], g.sm_scale, mass_correction)
-    r = rank_classes(sc, g.n8, g.nm, g.n4)
+    if g.tau > 0:
+        r = rank_adaptive(sc, g.n8, g.nm, g.n4, g.n4max, g.tau)
+    else:
+        r = rank_classes(sc, g.n8, g.nm, g.n4)
     return dict(scores=sc, **r)
 
 
