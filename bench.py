@@ -44,9 +44,10 @@ def executed_flops(w):
     N = w.F * ny * nx
     bs = w.ph * w.pw
     pm = getattr(w, "pct_mix", 0)
+    p4 = w.pct_fp4_max if getattr(w, "adapt_tau", 0.0) > 0 else w.pct_fp4   # the kernel runs the cap
     c8 = (w.pct_fp8 * N + 50) // 100
     c8m = ((w.pct_fp8 + pm) * N + 50) // 100
-    ck = ((w.pct_fp8 + pm + w.pct_fp4) * N + 50) // 100
+    ck = ((w.pct_fp8 + pm + p4) * N + 50) // 100
     rows = w.B * w.H * N
     per = 4.0 * bs * bs * w.d
     nm = c8m - c8
@@ -112,9 +113,10 @@ def draft_bytes(w) -> float:
     import math as _m
     N = w.F * _m.ceil(w.Hf / w.ph) * _m.ceil(w.Wf / w.pw)
     pm = getattr(w, "pct_mix", 0)
+    p4 = w.pct_fp4_max if getattr(w, "adapt_tau", 0.0) > 0 else w.pct_fp4
     c8 = (w.pct_fp8 * N + 50) // 100
     c8m = ((w.pct_fp8 + pm) * N + 50) // 100
-    ck = ((w.pct_fp8 + pm + w.pct_fp4) * N + 50) // 100
+    ck = ((w.pct_fp8 + pm + p4) * N + 50) // 100
     kept = max(c8, 1) + max(ck - c8m, 1) + (c8m - c8 if pm > 0 else 0)
     BH = w.B * w.H
     return float(BH * (4 * N * w.d * 4 + N * N + N * kept * 2))
@@ -517,7 +519,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_workloads and args.heads == 0:
         del ws, out
         others = {}
-        for name in ("wan480", "hunyuan720", "sweep0", "sweep1", "sweep2", "sweep3", "sweep4", "wan720mix"):
+        for name in ("wan480", "hunyuan720", "sweep0", "sweep1", "sweep2", "sweep3", "sweep4", "wan720mix",
+                     "wan720adapt"):
             if name == w.name:
                 continue
             wo = WORKLOADS[name]

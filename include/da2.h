@@ -69,6 +69,11 @@ typedef struct da2_config {
   int flags;            /* DA2_FLAG_* bits */
   int pct_mix;          /* percent of KV blocks in the mixed class (E4M3 scores, E2M1 P V),
                            ranked between FP8 and FP4; 0 gives the two-class path */
+  float adapt_tau;      /* > 0: error-bound-driven FP4 budget. Per query block, the KV blocks
+                           ranked after the fixed budgets join FP4, in rank order, while their
+                           draft score (estimated attention mass) is >= adapt_tau, up to
+                           pct_fp4_max percent FP4 blocks; 0 turns it off */
+  int pct_fp4_max;      /* the FP4 cap of the adaptive budget (>= pct_fp4) */
 } da2_config;
 
 enum {
@@ -130,7 +135,8 @@ typedef enum da2_status {
      tags     u8 [BH][N][N]  0 skip, 1 FP4, 2 FP8, 3 mixed for (query block, KV block).
      list8    i16 [BH][N][n8s], list4 i16 [BH][N][n4s], listm i16 [BH][N][nms]: kept KV
               blocks of each class per query block in ascending block order (n8s =
-              max(n8,1), n4s = max(n4,1), nms = max(nm,1)).
+              max(n8,1), n4s = max(n4max,1), nms = max(nm,1)); with the adaptive budget a
+              row's FP4 list holds its n4 .. n4max blocks followed by -1 entries.
      scores   fp32 [BH][N][N] (only with DA2_FLAG_EXPORT_SCORES, else size 0).
      err      u32 device error word (0 = no error). */
 typedef struct da2_views {
@@ -141,6 +147,7 @@ typedef struct da2_views {
   size_t tags, list8, list4, scores, err, total;
   int nm;               /* mixed KV blocks per query block */
   size_t listm;
+  int n4max;            /* FP4 list length (n4 unless the adaptive budget is on) */
 } da2_views;
 
 /* Workspace bytes needed for `cfg` (host only, no CUDA call). */

@@ -97,7 +97,7 @@ def geometry(w) -> Geometry:
     bs = w.ph * w.pw
     pm = getattr(w, "pct_mix", 0)
     n8, nm, n4 = budget_counts3(N, w.pct_fp8, pm, w.pct_fp4)
-    tau = float(getattr(w, "adapt_tau", 0.0))
+    tau = float(np.float32(getattr(w, "adapt_tau", 0.0)))      # a configuration value in fp32
     n4max = budget_counts3(N, w.pct_fp8, pm, w.pct_fp4_max)[2] if tau > 0 else n4
     sm = getattr(w, "sm_scale", 0.0) or 1.0 / math.sqrt(w.d)
     return Geometry(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, ny, nx, N, bs,
@@ -401,7 +401,7 @@ def rank_adaptive(scores, n8: int, nm: int, n4: int, n4max: int, tau: float):
     cnt = np.zeros(flat.shape[0], dtype=np.int64)
     j = np.arange(N)
     ck, ckmax = n8 + nm + n4, min(n8 + nm + n4max, N)
-    base4 = r["list4"].reshape(-1, n4)
+    base4 = r["list4"].reshape(flat.shape[0], n4)
     for row in range(flat.shape[0]):
         order = np.lexsort((j, -flat[row]))
         extra = [b for b in order[ck:ckmax] if flat[row, b] >= tau]

@@ -38,7 +38,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned
 class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "d", "F", "Hf", "Wf", "ph", "pw",
                                              "pct_fp8", "pct_fp4")] + \
-               [("sm_scale", ctypes.c_float), ("flags", ctypes.c_int), ("pct_mix", ctypes.c_int)]
+               [("sm_scale", ctypes.c_float), ("flags", ctypes.c_int), ("pct_mix", ctypes.c_int),
+                ("adapt_tau", ctypes.c_float), ("pct_fp4_max", ctypes.c_int)]
 
 
 _VIEW_INTS = ("N", "bs", "T", "Tp", "ny", "nx", "n8", "n4", "kv4")
@@ -50,7 +51,7 @@ _VIEW_SIZES = ("tile8_qk", "tile4_qk", "tile8_v", "tile4_v", "sf_qk", "sf_v",
 
 class Views(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in _VIEW_INTS] + [(n, ctypes.c_size_t) for n in _VIEW_SIZES] + \
-               [("nm", ctypes.c_int), ("listm", ctypes.c_size_t)]
+               [("nm", ctypes.c_int), ("listm", ctypes.c_size_t), ("n4max", ctypes.c_int)]
 
 
 class DA2Error(RuntimeError):
@@ -105,7 +106,8 @@ EXPORTED = ("da2_workspace_size", "da2_workspace_views", "da2_prepare", "da2_dra
 def config(w, flags: int = 0, sm_scale: float = 0.0) -> Config:
     """da2_config of a synth.Workload (or any object with the same fields)."""
     return Config(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, w.pct_fp8, w.pct_fp4,
-                  float(sm_scale), int(flags), int(getattr(w, "pct_mix", 0)))
+                  float(sm_scale), int(flags), int(getattr(w, "pct_mix", 0)),
+                  float(getattr(w, "adapt_tau", 0.0)), int(getattr(w, "pct_fp4_max", 0)))
 
 
 def _check(fn, st):
@@ -132,7 +134,7 @@ def workspace_size(cfg: Config) -> int:
 def workspace_views(cfg: Config) -> dict:
     v = Views()
     _check("da2_workspace_views", lib().da2_workspace_views(ctypes.byref(cfg), ctypes.byref(v)))
-    return {n: getattr(v, n) for n in _VIEW_INTS + _VIEW_SIZES + ("nm", "listm")}
+    return {n: getattr(v, n) for n in _VIEW_INTS + _VIEW_SIZES + ("nm", "listm", "n4max")}
 
 
 def prepare(cfg, q, k, v, ws, stream=None):

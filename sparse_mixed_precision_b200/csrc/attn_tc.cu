@@ -42,6 +42,8 @@
 // producer and the issuers stop issuing work, the producer waits for its copies in flight
 // and the issuers for their MMAs, the softmax warps run through the rest of their round
 // without waiting, and the kernel frees its tensor memory and exits.
+#include <type_traits>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -109,8 +111,9 @@ constexpr uint32_t kColP = 448;                                                 
 constexpr uint32_t kQ8 = 0, kQ4 = 16384, kSFQ = 24576, kQBytes = 25600;   // per tile
 constexpr uint32_t kStage0 = 2 * kQBytes;
 constexpr uint32_t kStK = 0, kStV = 16384, kStSFK = 32768, kStSFV = 33792, kStageBytes = 34816;
-constexpr uint32_t kMask = kStage0 + kStages * kStageBytes;   // 4 slot-validity masks x 4 words
-constexpr uint32_t kEdge = kMask + 64;             // edge class of every block (u8 [N <= 4096])
+constexpr uint32_t kMask = kStage0 + kStages * kStageBytes;   // 5 slot-validity masks x 4 words
+constexpr uint32_t kEdge = kMask + 128;            // edge class of every block (u8 [N <= 4096])
+constexpr int kNoBlock = 4;                        // mask class of a -1 list entry: no valid key
 constexpr uint32_t kBar = kEdge + 4096;
 constexpr uint32_t kSmemBytes = kBar + 256;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -194,8 +197,8 @@ __device__ __noinline__ void rescale_o(uint32_t taddr, float alpha) {
 // the block (checking here costs the loop several percent): after a timeout every later
 // wait returns at once, so the rest of the round runs through without waiting and the
 // warpgroup stops at the round's epilogue.
-template <int D, int BS>
-__device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileBars* tb, uint8_t* sm, uint32_t colP,
+template <int D, int BS, bool FP8>
+__device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t* sm, uint32_t colP,
                                               uint32_t tmem, uint32_t lane_base, uint32_t colO, int r,
                                               float c, int ecls, uint32_t gx, int t, float& m, float& l,
                                               unsigned long long wait_ns) {
@@ -233,8 +236,11 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
 #pragma unroll
   for (int q = 1; q < NG; ++q) mh = fmaxf(mh, gm[q]);
   const float m_new = fmaxf(m, mh * c);
-  const float alpha = ex2(m - m_new);
-  const float bias = kLog2_448 - m_new;
+  // a row whose blocks so far held no valid key keeps m = -inf: alpha 1, and the bias
+  // stays finite so that its p are 0
+  const bool none = m_new == -INFINITY;
+  const float alpha = none ? 1.0f : ex2(m - m_new);
+  const float bias = kLog2_448 - (none ? 0.0f : m_new);
   // The quantised P stays in registers until the exponential loop is done: only then does
   // the row wait for its tile's previous P V (which frees the P columns and O), so that
   // wait overlaps the loop.
@@ -247,7 +253,7 @@ __device__ __forceinline__ void softmax_block(const bool FP8, const Ws& w, TileB
   // row-sum partials: keys 4i+0/4i+1 in sA, 4i+2/4i+3 in sB
   f32x2 sA = pk2(0.0f, 0.0f), sB = pk2(0.0f, 0.0f);
   const f32x2 c2 = pk2(c, c);
-  if (FP8) {
+  if constexpr (FP8) {
     const f32x2 b2 = pk2(bias, bias);
     uint32_t wd[BS / 4];
 #pragma unroll
@@ -350,7 +356,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = g.N, BH = g.B * g.H;
   // phases: blocks t < n8 FP8, n8 <= t < n8m mixed (E4M3 scores, E2M1 P V), then FP4
-  const int n8 = g.n8, n8m = g.n8 + g.nm, nb = g.n8 + g.nm + g.n4;
+  // with the adaptive budget every row runs n4max FP4 entries; -1 entries are no block
+  // (a fully masked block that contributes nothing)
+  const int n8 = g.n8, n8m = g.n8 + g.nm, nb = g.n8 + g.nm + g.n4max;
   const int total = BH * N;
   constexpr int KV4 = BS < 64 ? 64 : BS;
   // work items of this CTA: blockIdx.x + m gridDim.x; round k takes m = 2k (A), 2k+1 (B)
@@ -390,13 +398,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       const int rem = n % (g.ny * g.nx), by = rem / g.nx, bx = rem - by * g.nx;
       ecl[n] = (uint8_t)(((by == g.ny - 1 && hl < g.ph) ? 2 : 0) | ((bx == g.nx - 1 && wl < g.pw) ? 1 : 0));
     }
-    if (tid < 16) {
+    if (tid < 20) {                                      // class 4 (no block) keeps no slot
       const int cls = tid >> 2, q = tid & 3;
       const int hv = (cls & 2) ? hl : g.ph, wv = (cls & 1) ? wl : g.pw;
       uint32_t bits = 0u;
       for (int e = 0; e < 32; ++e) {
         const int k = 32 * q + e, ky = k / g.pw, kx = k - ky * g.pw;
-        if (k < BS && ky < hv && kx < wv) bits |= 1u << e;
+        if (cls < kNoBlock && k < BS && ky < hv && kx < wv) bits |= 1u << e;
       }
       reinterpret_cast<uint32_t*>(sm + kMask)[tid] = bits;
     }
@@ -628,9 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
         continue;
       }
       const float sq = w.sq[qi];
-      const int16_t* l8 = w.list8 + qi * w.n8s;
-      const int16_t* lm = w.listm + qi * w.nms;
-      const int16_t* l4 = w.list4 + qi * w.n4s;
+
       float m = -INFINITY, l = 0.0f;
       // Block index j and key scale s_k[j] of every visited block, fetched 32 blocks at a
       // time (lane i holds block 32 ch + i) and broadcast by shuffles: the list entries of
@@ -638,13 +644,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
       // so no block waits on a global load.
       const float cq = sq * g.sm_scale * kLog2e;
       const float* skh = w.sk + (size_t)bh * N;
+      // list entries are fetched 32 blocks at a time; the three lists' addresses follow
+      // from the work item when needed (fewer live registers in the block loop)
       auto list_j = [&](int t) -> int {
-        const int j = t < nb ? (t < n8 ? l8[t] : (t < n8m ? lm[t - n8] : l4[t - n8m])) : 0;
-        return (j < 0 || j >= N) ? 0 : j;
+        int j = 0;
+        if (t < n8) j = w.list8[qi * w.n8s + t];
+        else if (t < n8m) j = w.listm[qi * w.nms + (t - n8)];
+        else if (t < nb) j = w.list4[qi * w.n4s + (t - n8m)];
+        return j < 0 ? -1 : (j >= N ? 0 : j);            // -1: no block
       };
       int jA = list_j(lane), jB = list_j(32 + lane), jC = list_j(64 + lane);
-      float sA = skh[jA], sB = skh[jB];
-      for (int t = 0; t < nb; ++t, ++gx) {
+      float sA = skh[jA < 0 ? 0 : jA], sB = skh[jB < 0 ? 0 : jB];
+      // one loop per P precision (FP8 blocks, then mixed and FP4 blocks), each with a
+      // single softmax body
+      auto step = [&](auto fp8, int t) {
         const int ln = t & 31;
         const int j = __shfl_sync(0xffffffffu, jA, ln);
         const float c = cq * __shfl_sync(0xffffffffu, sA, ln);
@@ -652,12 +665,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attention_tc(Geo g, Ws w, __nv_
           jA = jB;
           sA = sB;
           jB = jC;
-          sB = skh[jB];
+          sB = skh[jB < 0 ? 0 : jB];
           jC = list_j(t + 65 + lane);
         }
-        const int ecls = sm[kEdge + j];
-        softmax_block<D, BS>(t < n8, w, tb, sm, colP, tmem, lane_base, colO, r, c, ecls, gx, t, m, l, g.wait_ns);
-      }
+        const int ecls = j < 0 ? kNoBlock : sm[kEdge + j];
+        softmax_block<D, BS, decltype(fp8)::value>(w, tb, sm, colP, tmem, lane_base, colO, r, c, ecls, gx, t, m,
+                                                     l, g.wait_ns);
+      };
+      int t = 0;
+      for (; t < n8; ++t, ++gx) step(std::true_type{}, t);
+      for (; t < nb; ++t, ++gx) step(std::false_type{}, t);
       // ---- epilogue: O / l, V channel scale, bf16, original token order ----
       if (!wait_bar(&tb->o_full, k & 1, w.err, g.wait_ns)) {
         dead = true;

@@ -16,6 +16,8 @@ struct Geo {
   int B, H, d, F, Hf, Wf, ph, pw;
   int ny, nx, N, bs, T, Tp, n8, n4, kv4;
   int nm;     // mixed KV blocks per query block (E4M3 scores, E2M1 P V)
+  int n4max;  // FP4 list length per query block (n4 unless the adaptive budget is on)
+  float tau;  // adaptive FP4 budget threshold on the draft score (0: off)
   float sm_scale;
   int flags;
   int bthd;   // q, k, v, out token-major [B,T,H,d] instead of [B,H,T,d]

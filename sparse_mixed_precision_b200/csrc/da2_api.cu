@@ -29,6 +29,10 @@ da2_status check_config(const da2_config* c) {
   if (c->pct_fp8 < 0 || c->pct_fp4 < 0 || c->pct_mix < 0 || c->pct_fp8 + c->pct_mix + c->pct_fp4 > 100)
     return DA2_ERR_INVALID_ARG;
   if (!(c->sm_scale >= 0.0f) || std::isinf(c->sm_scale)) return DA2_ERR_INVALID_ARG;
+  if (!(c->adapt_tau >= 0.0f) || std::isinf(c->adapt_tau)) return DA2_ERR_INVALID_ARG;
+  if (c->adapt_tau > 0.0f &&
+      (c->pct_fp4_max < c->pct_fp4 || c->pct_fp8 + c->pct_mix + c->pct_fp4_max > 100))
+    return DA2_ERR_INVALID_ARG;
   if (c->flags & ~(DA2_FLAG_EXPORT_SCORES | DA2_FLAG_NO_MASS_CORRECTION | DA2_FLAG_LAYOUT_BTHD |
                    DA2_FLAG_TEST_STALL))
     return DA2_ERR_INVALID_ARG;
@@ -56,6 +60,9 @@ void fill_views(const da2_config* c, da2_views* v) {
   v->n8 = c8;
   v->nm = c8m - c8;
   v->n4 = ck - c8m;
+  v->n4max = c->adapt_tau > 0.0f
+                 ? ((c->pct_fp8 + c->pct_mix + c->pct_fp4_max) * v->N + 50) / 100 - c8m
+                 : v->n4;
   v->kv4 = v->bs < 64 ? 64 : v->bs;
   const size_t d = c->d, bs = v->bs, N = v->N, BH = (size_t)c->B * c->H;
   v->tile8_qk = bs * d;
@@ -64,7 +71,7 @@ void fill_views(const da2_config* c, da2_views* v) {
   v->tile4_v = d * v->kv4 / 2;
   v->sf_qk = (d / 64) * 512;
   v->sf_v = (v->kv4 / 64) * 512;
-  const size_t n8s = v->n8 > 0 ? v->n8 : 1, n4s = v->n4 > 0 ? v->n4 : 1, nms = v->nm > 0 ? v->nm : 1;
+  const size_t n8s = v->n8 > 0 ? v->n8 : 1, n4s = v->n4max > 0 ? v->n4max : 1, nms = v->nm > 0 ? v->nm : 1;
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + bytes); return o; };
   v->q8 = take(BH * N * v->tile8_qk);
@@ -98,6 +105,8 @@ Geo make_geo(const da2_config* c, const da2_views& v) {
   g.B = c->B; g.H = c->H; g.d = c->d; g.F = c->F; g.Hf = c->Hf; g.Wf = c->Wf;
   g.ph = c->ph; g.pw = c->pw; g.ny = v.ny; g.nx = v.nx; g.N = v.N; g.bs = v.bs;
   g.T = v.T; g.Tp = v.Tp; g.n8 = v.n8; g.n4 = v.n4; g.kv4 = v.kv4; g.nm = v.nm;
+  g.n4max = v.n4max;
+  g.tau = c->adapt_tau;
   g.sm_scale = c->sm_scale > 0.0f ? c->sm_scale : 1.0f / std::sqrt((float)c->d);
   g.flags = c->flags;
   g.bthd = (c->flags & DA2_FLAG_LAYOUT_BTHD) ? 1 : 0;
@@ -129,7 +138,7 @@ Ws make_ws(void* base, const da2_views& v) {
   w.tile8_qk = v.tile8_qk; w.tile4_qk = v.tile4_qk; w.tile8_v = v.tile8_v; w.tile4_v = v.tile4_v;
   w.sf_qk = v.sf_qk; w.sf_v = v.sf_v;
   w.n8s = v.n8 > 0 ? v.n8 : 1;
-  w.n4s = v.n4 > 0 ? v.n4 : 1;
+  w.n4s = v.n4max > 0 ? v.n4max : 1;
   w.nms = v.nm > 0 ? v.nm : 1;
   return w;
 }

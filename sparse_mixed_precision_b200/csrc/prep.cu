@@ -248,29 +248,44 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
     uint8_t* t8 = w.v8 + ((size_t)bh * g.N + n) * w.tile8_v;
     uint8_t* t4 = w.v4 + ((size_t)bh * g.N + n) * w.tile4_v;
     const int SC = bs / 16, SC4 = g.kv4 / 16;
-    for (int u = tid; u < D * SC4; u += 256) {
-      const int cg = u / (8 * SC4), within = u - cg * 8 * SC4;
-      const int sc = within >> 3, cc = within & 7;
-      const int c = cg * 8 + cc;
-      const float inv = vinv[c];
-      float y[16];
+    // one unit = channels c, c + 1 of one 16-slot group; a warp takes 32 consecutive channel
+    // pairs of one group, so its 32-bit reads cover 128 contiguous bytes of each staged row
+    constexpr int CP = D / 2;
+    for (int u = tid; u < CP * SC4; u += 256) {
+      const int sc = u / CP, c = 2 * (u - sc * CP);
+      const float inv0 = vinv[c], inv1 = vinv[c + 1];
+      float y0[16], y1[16];
       if (sc < SC) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(__bfloat162float(X[(sc * 16 + i) * RS + c]), inv);
-        uint32_t p8[4];
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t pr = *reinterpret_cast<const uint32_t*>(X + (sc * 16 + i) * RS + c);
+          y0[i] = __fmul_rn(__uint_as_float(pr << 16), inv0);
+          y1[i] = __fmul_rn(__uint_as_float(pr & 0xFFFF0000u), inv1);
+        }
+        uint32_t p8[4], q8[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          p8[i] = (uint32_t)f32x2_to_e4m3x2(y[4 * i], y[4 * i + 1]) |
-                  ((uint32_t)f32x2_to_e4m3x2(y[4 * i + 2], y[4 * i + 3]) << 16);
+        for (int i = 0; i < 4; ++i) {
+          p8[i] = (uint32_t)f32x2_to_e4m3x2(y0[4 * i], y0[4 * i + 1]) |
+                  ((uint32_t)f32x2_to_e4m3x2(y0[4 * i + 2], y0[4 * i + 3]) << 16);
+          q8[i] = (uint32_t)f32x2_to_e4m3x2(y1[4 * i], y1[4 * i + 1]) |
+                  ((uint32_t)f32x2_to_e4m3x2(y1[4 * i + 2], y1[4 * i + 3]) << 16);
+        }
         *reinterpret_cast<uint4*>(t8 + kmajor_off(c, sc * 16, bs)) = make_uint4(p8[0], p8[1], p8[2], p8[3]);
+        *reinterpret_cast<uint4*>(t8 + kmajor_off(c + 1, sc * 16, bs)) = make_uint4(q8[0], q8[1], q8[2], q8[3]);
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+          y0[i] = 0.0f;
+          y1[i] = 0.0f;
+        }
       }
       uint32_t p4[2];
-      const uint8_t s4 = quant_fp4_group16_tab(y, p4, rcp_tab);
+      const uint8_t s40 = quant_fp4_group16_tab(y0, p4, rcp_tab);
       *reinterpret_cast<uint2*>(t4 + kmajor_off(c, sc * 8, g.kv4 / 2)) = make_uint2(p4[0], p4[1]);
-      sfbuf[sf_off(sc >> 2, c, sc & 3)] = s4;
+      const uint8_t s41 = quant_fp4_group16_tab(y1, p4, rcp_tab);
+      *reinterpret_cast<uint2*>(t4 + kmajor_off(c + 1, sc * 8, g.kv4 / 2)) = make_uint2(p4[0], p4[1]);
+      sfbuf[sf_off(sc >> 2, c, sc & 3)] = s40;
+      sfbuf[sf_off(sc >> 2, c + 1, sc & 3)] = s41;
     }
     __syncthreads();
     uint8_t* sfo = w.sfv4 + ((size_t)bh * g.N + n) * w.sf_v;

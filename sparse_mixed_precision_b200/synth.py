@@ -62,6 +62,10 @@ WORKLOADS = {
 }
 # The 720p layer with the mixed class between FP8 and FP4 (FP8 10 / mixed 10 / FP4 20 / skip 60).
 WORKLOADS["wan720mix"] = Workload("wan720mix", 1, 40, 128, 21, 45, 80, 8, 16, 10, 20, 4, False, 1002, 10)
+# The 720p layer with the error-bound-driven FP4 budget: FP8 10 / FP4 20, skipped blocks
+# whose draft score reaches 0.002 recovered at FP4 up to 40 %.
+WORKLOADS["wan720adapt"] = Workload("wan720adapt", 1, 40, 128, 21, 45, 80, 8, 16, 10, 20, 4, False, 1002, 0,
+                                    0.002, 40)
 SWEEP_BUDGETS = [(100, 0), (0, 100), (25, 0), (10, 30), (5, 45)]
 for _i, (_p8, _p4) in enumerate(SWEEP_BUDGETS):
     WORKLOADS[f"sweep{_i}"] = Workload(f"sweep{_i}", 2, 40, 128, 21, 45, 80, 8, 16,

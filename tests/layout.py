@@ -90,10 +90,11 @@ class WsReader:
 
     def lists(self, bh0, bh1):
         v = self.v
-        n8s, n4s = max(v["n8"], 1), max(v["n4"], 1)
+        n4 = v.get("n4max", v["n4"])                # the FP4 list's length (adaptive budget)
+        n8s, n4s = max(v["n8"], 1), max(n4, 1)
         l8 = self._bytes("list8", bh0, bh1, v["N"] * n8s * 2).view(np.int16).reshape(bh1 - bh0, v["N"], n8s)
         l4 = self._bytes("list4", bh0, bh1, v["N"] * n4s * 2).view(np.int16).reshape(bh1 - bh0, v["N"], n4s)
-        return l8[..., : v["n8"]].astype(np.int64), l4[..., : v["n4"]].astype(np.int64)
+        return l8[..., : v["n8"]].astype(np.int64), l4[..., :n4].astype(np.int64)
 
     def listm(self, bh0, bh1):
         v = self.v

@@ -144,3 +144,16 @@ def test_mixed_budget_counts_and_limits():
     assert L.da2_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == 1
     neg = da2.config(scaled(WORKLOADS["tiny"], pct_mix=-1))
     assert L.da2_workspace_size(ctypes.byref(neg), ctypes.byref(n)) == 1
+
+
+def test_adaptive_budget_views_and_limits():
+    L = da2.lib()
+    n = ctypes.c_size_t()
+    w = scaled(WORKLOADS["wan720"], pct_fp8=10, pct_fp4=20, pct_fp4_max=40, adapt_tau=0.002)
+    v = da2.workspace_views(da2.config(w))
+    assert (v["n8"], v["n4"], v["n4max"]) == (63, 126, 252)       # cuts 63, 189, 315
+    assert da2.workspace_views(da2.config(WORKLOADS["wan720"]))["n4max"] == 189
+    for bad in (dict(pct_fp4_max=10, adapt_tau=0.01), dict(pct_fp4_max=90, adapt_tau=0.01),
+                dict(pct_fp4_max=50, adapt_tau=-1.0), dict(pct_fp4_max=50, adapt_tau=float("inf"))):
+        cfg = da2.config(scaled(WORKLOADS["tiny"], **bad))
+        assert L.da2_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 1, bad

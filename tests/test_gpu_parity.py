@@ -330,3 +330,51 @@ def test_mixed_class_parity(name, kw):
             [0, g.N - 1] + list(np.random.default_rng(h).choice(g.N, 6, replace=False))))
         check_attention(w, views, P, l8[0], l4[0], out[0, h].float().cpu().numpy(), blocks, g, lm=lm[0])
     assert torch.isfinite(out).all()
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", dict(pct_fp8=10, pct_fp4=15, pct_fp4_max=45, adapt_tau=0.01)),
+    ("tiny", dict(pct_fp8=0, pct_fp4=0, pct_fp4_max=30, adapt_tau=0.02)),
+    ("wan720", dict(H=3, F=3, pct_fp8=10, pct_mix=5, pct_fp4=15, pct_fp4_max=35, adapt_tau=0.004)),
+], ids=["tiny-adaptive", "tiny-adaptive-from-zero", "wan720-adaptive-mixed"])
+def test_adaptive_budget_parity(name, kw):
+    # error-bound-driven FP4 budget: the CUDA fp32 scores ranked by the oracle's adaptive
+    # rule give exactly the CUDA tags and padded lists; against the oracle's fp64 scores a
+    # tag may differ only for a block within 1e-5 x (row max) of a rank cut or of the
+    # threshold; outputs within the tolerance (padding entries contribute nothing)
+    w = scaled(WORKLOADS[name], **kw)
+    q, k, v = generate(w, device="cuda")
+    cfg, views, ws, out = run_cuda(w, q, k, v)
+    rd = WsReader(ws, views, w.d)
+    g = O.geometry(scaled(w, B=1, H=1))
+    assert views["n4max"] == g.n4max > g.n4
+    recovered = 0
+    for h in range(w.H):
+        qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+        P = check_prep(w, views, rd, h, qh, kh, vh)
+        tags = rd.tags(h, h + 1)[0]
+        l8, l4 = rd.lists(h, h + 1)
+        lm = rd.listm(h, h + 1) if g.nm > 0 else None
+        sc = rd.scores(h, h + 1)[0].astype(np.float64)
+        r2 = O.rank_adaptive(sc, g.n8, g.nm, g.n4, g.n4max, g.tau)
+        assert np.array_equal(r2["tags"], tags) and np.array_equal(r2["list8"], l8[0])
+        assert np.array_equal(r2["list4"], l4[0])
+        if lm is not None:
+            assert np.array_equal(r2["listm"], lm[0])
+        recovered += int((r2["count4"] - g.n4).sum())
+        sel = O.draft_select(P)
+        ref = sel["scores"][0, 0]
+        for r in np.flatnonzero((tags != sel["tags"][0, 0]).any(axis=1)):
+            order = np.lexsort((np.arange(g.N), -ref[r]))
+            cuts = [ref[r, order[c]] for c in range(g.N)
+                    if c in (g.n8 - 1, g.n8, g.n8 + g.nm - 1, g.n8 + g.nm, g.n8 + g.nm + g.n4 - 1,
+                             g.n8 + g.nm + g.n4, g.n8 + g.nm + g.n4max - 1, g.n8 + g.nm + g.n4max)]
+            cuts.append(g.tau)
+            for j in np.flatnonzero(tags[r] != sel["tags"][0, 0, r]):
+                assert min(abs(ref[r, j] - c) for c in cuts) <= 1e-5 * ref[r].max(), (r, j)
+        blocks = list(range(g.N)) if g.N <= 64 else sorted(set(
+            [0, g.N - 1] + list(np.random.default_rng(h).choice(g.N, 6, replace=False))))
+        check_attention(w, views, P, l8[0], l4[0], out[0, h].float().cpu().numpy(), blocks, g,
+                        lm=None if lm is None else lm[0])
+    assert recovered > 0                                         # the rule did recover blocks
+    assert torch.isfinite(out).all()

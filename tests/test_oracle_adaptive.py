@@ -28,12 +28,15 @@ def test_threshold_extremes_reduce_to_fixed_budgets():
     assert np.array_equal(lo["tags"], t2) and np.array_equal(lo["list4"], l42)
 
 
-def test_recovered_blocks_brute_force():
+import pytest
+
+
+@pytest.mark.parametrize("n8,nm,n4,n4max,tau", [(6, 4, 10, 30, 0.012), (0, 0, 0, 20, 0.02)])
+def test_recovered_blocks_brute_force(n8, nm, n4, n4max, tau):
     rng = np.random.default_rng(4)
     N = 64
     sc = rng.random((20, N)) ** 3
     sc /= sc.sum(axis=1, keepdims=True)
-    n8, nm, n4, n4max, tau = 6, 4, 10, 30, 0.012
     r = O.rank_adaptive(sc, n8, nm, n4, n4max, tau)
     for row in range(sc.shape[0]):
         order = sorted(range(N), key=lambda j: (-sc[row, j], j))
