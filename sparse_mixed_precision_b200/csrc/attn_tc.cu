@@ -208,7 +208,7 @@ __device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t
   tc::fence_after_sync();
   uint32_t sr[BS];
 #pragma unroll
-  for (int c0 = 0; c0 < BS; c0 += 16) tc::tmem_ld16(tmem + lane_base + kColS + c0, sr + c0);
+  for (int c0 = 0; c0 < BS; c0 += 32) tc::tmem_ld32(tmem + lane_base + kColS + c0, sr + c0);
 #pragma unroll
   for (int c0 = 0; c0 < BS; c0 += 16) tc::tmem_wait_ld16(sr + c0);
   tc::fence_before_sync();
@@ -270,8 +270,13 @@ __device__ __forceinline__ void softmax_block(const Ws& w, TileBars* tb, uint8_t
       }
     }
     wait_p_free();
+    if constexpr (NG >= 4) {
 #pragma unroll
-    for (int q = 0; q < NG; ++q) tc::tmem_st4(tmem + lane_base + colP + 4 * q, wd + 4 * q);
+      for (int q = 0; q < NG; q += 4) tc::tmem_st16(tmem + lane_base + colP + 4 * q, wd + 4 * q);
+    } else {
+#pragma unroll
+      for (int q = 0; q < NG; ++q) tc::tmem_st4(tmem + lane_base + colP + 4 * q, wd + 4 * q);
+    }
   } else {
     uint32_t sfw[KV4 / 64];
 #pragma unroll
