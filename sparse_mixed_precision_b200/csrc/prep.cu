@@ -77,6 +77,40 @@ __global__ void __launch_bounds__(256) k_vamax(Geo g, const __nv_bfloat16* __res
   }
 }
 
+// Pairs of fp32 values for the packed f32x2 multiply (each lane rounded as fmul.rn).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// y[i] * s for 16 values, two per packed multiply.
+__device__ __forceinline__ void scale16(const float* x, float s, float* y) {
+  const f32x2 s2 = pk2(s, s);
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) upk2(mul2(pk2(x[i], x[i + 1]), s2), y[i], y[i + 1]);
+}
+
+// a / 6 correctly rounded for finite a >= 0, in three FMA-pipe steps: q0 = a * fl(1/6), the
+// exact residual r = a - 6 q0 (one fma), q = q0 + r * fl(1/6). The quotient a / 6 = (a / 2) / 3
+// lies, in units of its own ulp, at a fraction 0, 1/3 or 2/3 from the fp32 grid, never
+// within the correction's residual error of a rounding midpoint, so q equals the IEEE
+// quotient (values below 2^-126 only reach E4M3 code 0 either way).
+__device__ __forceinline__ float div6_rn(float a) {
+  const float c = 0.16666667163372040f;       // fl(1/6)
+  const float q0 = __fmul_rn(a, c);
+  const float r = __fmaf_rn(-6.0f, q0, a);
+  return __fmaf_rn(r, c, q0);
+}
+
 // Quantise one group of 16 values y (already divided by their outer scale) to E2M1 with an
 // E4M3 group scale: sigma = E4M3(amax16 / 6); codes = E2M1(y * (1/sigma)), the correctly
 // rounded reciprocal taken from a table over the 128 non-negative E4M3 codes (filled with
@@ -87,12 +121,11 @@ __device__ __forceinline__ uint8_t quant_fp4_group16_tab(const float* y, uint32_
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[i]));
-  const uint8_t sc = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+  const uint8_t sc = f32_to_e4m3(div6_rn(amax));
   if (sc != 0) {
     const float r = rcp_tab[sc & 0x7F];
     float z[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) z[i] = __fmul_rn(y[i], r);
+    scale16(y, r, z);
     packed2[0] = f32x8_to_e2m1x8(z);
     packed2[1] = f32x8_to_e2m1x8(z + 8);
   } else {
@@ -218,8 +251,7 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
       float xf[16];
       bf16x8_to_f32(*reinterpret_cast<const uint4*>(X + r * RS + kc * 16), xf);
       bf16x8_to_f32(*reinterpret_cast<const uint4*>(X + r * RS + kc * 16 + 8), xf + 8);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(xf[i], inv);
+      scale16(xf, inv, y);
       uint32_t p8[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -259,8 +291,8 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint32_t pr = *reinterpret_cast<const uint32_t*>(X + (sc * 16 + i) * RS + c);
-          y0[i] = __fmul_rn(__uint_as_float(pr << 16), inv0);
-          y1[i] = __fmul_rn(__uint_as_float(pr & 0xFFFF0000u), inv1);
+          upk2(mul2(pk2(__uint_as_float(pr << 16), __uint_as_float(pr & 0xFFFF0000u)), pk2(inv0, inv1)),
+               y0[i], y1[i]);
         }
         uint32_t p8[4], q8[4];
 #pragma unroll

@@ -378,3 +378,40 @@ def test_adaptive_budget_parity(name, kw):
                         lm=None if lm is None else lm[0])
     assert recovered > 0                                         # the rule did recover blocks
     assert torch.isfinite(out).all()
+
+
+def test_no_mass_correction_and_explicit_softmax_scale():
+    # DA2_FLAG_NO_MASS_CORRECTION drops the ln(valid tokens) term of the draft logits and an
+    # explicit sm_scale replaces 1/sqrt(d): both change the ranking and the attention; the
+    # windows here are short at both edges, so the dropped term matters
+    import types
+    w = scaled(WORKLOADS["tiny"], F=2, Hf=13, Wf=29, name="tiny-edges-nomass")
+    sm = 0.09
+    q, k, v = generate(w, device="cuda")
+    cfg = da2.config(w, flags=da2.FLAG_EXPORT_SCORES | da2.FLAG_NO_MASS_CORRECTION, sm_scale=sm)
+    views = da2.workspace_views(cfg)
+    ws = torch.empty(views["total"], dtype=torch.uint8, device="cuda")
+    out = torch.full_like(q, float("nan"))
+    da2.forward(cfg, q, k, v, out, ws)
+    torch.cuda.synchronize()
+    assert da2.get_error(cfg, ws) == 0
+    rd = WsReader(ws, views, w.d)
+    wo = types.SimpleNamespace(**scaled(w, B=1, H=1).as_dict(), sm_scale=sm)
+    g = O.geometry(wo)
+    assert g.sm_scale == sm
+    moved = 0
+    for h in range(w.H):
+        qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+        P = O.prepare(wo, qh, kh, vh)
+        sel = O.draft_select(P, mass_correction=False)
+        sel_mass = O.draft_select(P, mass_correction=True)
+        tags = rd.tags(h, h + 1)[0]
+        l8, l4 = rd.lists(h, h + 1)
+        sc = rd.scores(h, h + 1)[0].astype(np.float64)
+        t2, a8, a4 = O.rank(sc, g.n8, g.n4)
+        assert np.array_equal(t2, tags) and np.array_equal(a8, l8[0]) and np.array_equal(a4, l4[0])
+        ref = sel["scores"][0, 0]
+        assert np.abs(sc - ref).max() <= 1e-5 * ref.max()          # the uncorrected scores
+        moved += int((sel["tags"] != sel_mass["tags"]).sum())
+        check_attention(w, views, P, l8[0], l4[0], out[0, h].float().cpu().numpy(), list(range(g.N)), g)
+    assert moved > 0                                               # the flag changed the ranking
