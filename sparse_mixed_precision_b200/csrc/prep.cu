@@ -30,6 +30,33 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 u, float* f) {
   }
 }
 
+// 16-byte global -> shared copy that bypasses L1 (cp.async.cg); src_bytes 0 writes zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// lo += bf16 low half of w, hi += bf16 high half, each one fp32 add rounded to nearest (the
+// bf16 operand widens exactly, so this is the fp32 sum of the widened values).
+__device__ __forceinline__ void acc_bf16x2(uint32_t w, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+      : "+f"(lo), "+f"(hi) : "r"(w));
+}
+// Elementwise max / min of two bf16 pairs (exact; a NaN operand yields the other).
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // ---- K0: amax of V over all tokens, per (b, h, channel) ----
 // grid (chunks, B*H); vamax must be zero on entry (non-negative floats compare as uints).
 // BTHD: q, k, v token-major [B,T,H,d] (token stride H*D) instead of [B,H,T,d] (stride D).
@@ -169,17 +196,16 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
     int s0 = tid / VPR;
     int wy = s0 / g.pw, wx = s0 - wy * g.pw;
     const int dy = DS / g.pw, dx = DS - dy * g.pw;
+    // every copy of the thread in flight at once; padded slots are zero-filled
     for (int sl = s0; sl < bs; sl += DS) {
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (wy < hv && wx < wv) {
-        const size_t t = (size_t)f * g.Hf * g.Wf + (size_t)(y0 + wy) * g.Wf + (x0 + wx);
-        val = ld_stream_u4(sbase + t * ts + cv * 8);
-      }
-      *reinterpret_cast<uint4*>(X + sl * RS + cv * 8) = val;
+      const bool ok = wy < hv && wx < wv;
+      const size_t t = ok ? (size_t)f * g.Hf * g.Wf + (size_t)(y0 + wy) * g.Wf + (x0 + wx) : 0;
+      cp_async16(X + sl * RS + cv * 8, sbase + t * ts + cv * 8, ok ? 16u : 0u);
       wx += dx;
       wy += dy;
       if (wx >= g.pw) { wx -= g.pw; ++wy; }
     }
+    cp_async_wait_all();
   }
   const int sfbytes = which < 2 ? (int)w.sf_qk : (int)w.sf_v;
   for (int i = tid; i < sfbytes / 4; i += 256) reinterpret_cast<uint32_t*>(sfbuf)[i] = 0u;
@@ -187,55 +213,83 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
   __syncthreads();
 
   if (which < 2) {
-    // ---- draft pooling: fp32 running sum in slot order, then IEEE divide; exact max ----
-    // threads [0, D/2): sums of channel pairs; [D/2, D): maxima of channel pairs
+    // ---- draft pooling and block amax ----
+    // Warps [0, NSW): fp32 running sums in slot order (two channels per lane), then an IEEE
+    // divide by the number of valid tokens. Warps [NSW, 8): exact maxima and minima as bf16
+    // pairs, 16 bytes of channels per lane, the valid slots split into G interleaved groups;
+    // the block amax is the largest |max| or |min| (padded zero slots cannot raise it).
+    constexpr int NSW = D / 64, CPW = D / 8, SPW = 32 / CPW, NMW = 8 - NSW, G = NMW * SPW;
     float* avg_out = (which == 0 ? w.qavg : w.kavg) + ((size_t)bh * g.N + n) * D;
     float* max_out = (which == 0 ? w.qmax : w.kmax) + ((size_t)bh * g.N + n) * D;
-    if (tid < D) {
-      const bool do_sum = tid < D / 2;
-      const int c2 = 2 * (tid % (D / 2));
-      float a0 = do_sum ? 0.0f : -INFINITY, a1 = a0;
+    uint32_t* pmax = reinterpret_cast<uint32_t*>(rcp_tab + 128);   // [NMW][CPW][4]
+    float* wam = reinterpret_cast<float*>(pmax + NMW * CPW * 4);    // [NMW]
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < NSW) {
+      const int c2 = 2 * (warp * 32 + lane);
+      float a0 = 0.0f, a1 = 0.0f;
       for (int wy = 0; wy < hv; ++wy) {
         const __nv_bfloat16* row = X + wy * g.pw * RS + c2;
-        if (do_sum) {
 #pragma unroll 4
-          for (int wx = 0; wx < wv; ++wx) {
-            const uint32_t u = *reinterpret_cast<const uint32_t*>(row + wx * RS);
-            a0 = __fadd_rn(a0, __uint_as_float(u << 16));
-            a1 = __fadd_rn(a1, __uint_as_float(u & 0xFFFF0000u));
+        for (int wx = 0; wx < wv; ++wx) acc_bf16x2(*reinterpret_cast<const uint32_t*>(row + wx * RS), a0, a1);
+      }
+      const float cnt = (float)(hv * wv);
+      *reinterpret_cast<float2*>(avg_out + c2) = make_float2(__fdiv_rn(a0, cnt), __fdiv_rn(a1, cnt));
+    } else {
+      const int mw = warp - NSW, ch = lane % CPW, sg = mw * SPW + lane / CPW;
+      uint32_t mx[4], mn[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mx[i] = 0xFF80FF80u;                                       // -inf pairs
+        mn[i] = 0x7F807F80u;                                       // +inf pairs
+      }
+      bool any = false;
+      int wy = sg / g.pw, wx = sg - wy * g.pw;
+      const int dy = G / g.pw, dx = G - dy * g.pw;
+      for (int sl = sg; sl < bs; sl += G) {
+        if (wy < hv && wx < wv) {
+          const uint4 u = *reinterpret_cast<const uint4*>(X + sl * RS + ch * 8);
+          const uint32_t e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            mx[i] = bmax2(mx[i], e[i]);
+            mn[i] = bmin2(mn[i], e[i]);
           }
-        } else {
-#pragma unroll 4
-          for (int wx = 0; wx < wv; ++wx) {
-            const uint32_t u = *reinterpret_cast<const uint32_t*>(row + wx * RS);
-            a0 = fmaxf(a0, __uint_as_float(u << 16));
-            a1 = fmaxf(a1, __uint_as_float(u & 0xFFFF0000u));
-          }
+          any = true;
         }
+        wx += dx;
+        wy += dy;
+        if (wx >= g.pw) { wx -= g.pw; ++wy; }
       }
-      if (do_sum) {
-        const float cnt = (float)(hv * wv);
-        *reinterpret_cast<float2*>(avg_out + c2) = make_float2(__fdiv_rn(a0, cnt), __fdiv_rn(a1, cnt));
-      } else {
-        *reinterpret_cast<float2*>(max_out + c2) = make_float2(a0, a1);
+      uint32_t a2 = 0u;                                            // |x| maxima as bf16 pairs
+      if (any) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a2 = bmax2(a2, bmax2(mx[i] & 0x7FFF7FFFu, mn[i] & 0x7FFF7FFFu));
       }
-    }
-    // ---- block amax -> outer scale ----
-    float am = 0.0f;
-    for (int u = tid; u < bs * VPR; u += 256) {
-      const int s = u / VPR, cv = u - s * VPR;
-      float fv[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(X + s * RS + cv * 8), fv);
+      float am = fmaxf(__uint_as_float(a2 << 16), __uint_as_float(a2 & 0xFFFF0000u));
 #pragma unroll
-      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(fv[i]));
-    }
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-    if ((tid & 31) == 0) red[tid >> 5] = am;
+      for (int o = CPW; o < 32; o <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = bmax2(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o));
+      }
+      if (lane < CPW) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pmax[(mw * CPW + ch) * 4 + i] = mx[i];
+      }
+      if (lane == 0) wam[mw] = am;
+    }
     __syncthreads();
-    am = red[0];
+    if (tid < D / 2) {                                             // channel pair 2 tid, 2 tid + 1
+      uint32_t m2 = pmax[tid];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) am = fmaxf(am, red[i]);
+      for (int k = 1; k < NMW; ++k) m2 = bmax2(m2, pmax[k * CPW * 4 + tid]);
+      *reinterpret_cast<float2*>(max_out + 2 * tid) =
+          make_float2(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+    }
+    float am = wam[0];
+#pragma unroll
+    for (int k = 1; k < NMW; ++k) am = fmaxf(am, wam[k]);
     const float inv = am > 0.0f ? __fdiv_rn(kE4M3Max, am) : 1.0f;
     if (tid == 0) (which == 0 ? w.sq : w.sk)[(size_t)bh * g.N + n] = am > 0.0f ? __fdiv_rn(am, kE4M3Max) : 1.0f;
 
@@ -327,7 +381,8 @@ __global__ void __launch_bounds__(256) k_prepare(Geo g, Ws w, const __nv_bfloat1
 }
 
 size_t prepare_smem_bytes(const Geo& g) {
-  return (size_t)g.bs * (g.d + 8) * 2 + 1024 + 4 * 128 + 4 * 128;
+  // staged window, group scales, reduction scratch, E4M3 reciprocals, pooled maxima
+  return (size_t)g.bs * (g.d + 8) * 2 + 1024 + 4 * 128 + 4 * 128 + 4 * (8 * 16 * 4 + 8);
 }
 
 cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
