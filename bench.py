@@ -29,7 +29,7 @@ from sparse_mixed_precision_b200.synth import WORKLOADS, generate  # noqa: E402
 
 METRIC = "dense-equivalent TFLOP/s of one DraftAttention2 attention call (75.6k tokens)"
 UNIT = "TFLOP/s"
-KERNELS_PER_STEP = 4      # k_vamax, k_prepare, k_draft_select, attention
+KERNELS_PER_STEP = 4      # k_prepare_qk, k_prepare_v, draft selection, attention
 
 
 def dense_flops(w) -> float:
