@@ -234,11 +234,13 @@ __global__ void __launch_bounds__(kDraftThreads) k_draft_select(Geo g, Ws w, int
 }
 
 // Register-tiled draft logits for up to 1024 key blocks: a CTA of KL = blockDim.x threads
-// takes 16 query blocks of one (b, h); thread t owns key blocks t and t + KL, all 16 query
-// rows and both maps, as packed pairs of rows (f32x2 FMA). The pooled queries sit in shared
-// memory transposed ([map][channel][row], read as float4 by every thread alike); each thread
-// streams its own two pooled key rows (16-byte loads through L1). Then the same per-row
-// ranking as the general kernel.
+// takes 16 query blocks of one (b, h); thread t owns key blocks t and t + KL and all 16 query
+// rows, one map after the other, as packed pairs of rows (f32x2 FMA). The pooled queries sit
+// in shared memory transposed ([map][channel][row], read as float4 by every thread alike);
+// each thread streams its own two pooled key rows (16-byte loads through L1). Then the same
+// per-row ranking as the general kernel. At 64 registers a thread and about 111 KB of
+// shared memory (up to 630 key blocks) two CTAs share an SM, so that the latency of one
+// CTA's phases is hidden by the other's warps.
 constexpr int kTileRows = 16;
 
 __device__ __forceinline__ unsigned long long pk2f(float lo, float hi) {
@@ -257,7 +259,7 @@ __device__ __forceinline__ unsigned long long fma2f(unsigned long long a, unsign
 }
 
 template <int D>
-__global__ void __launch_bounds__(kDraftThreads, 1) k_draft_tiled(Geo g, Ws w) {
+__global__ void __launch_bounds__(kDraftThreads, 2) k_draft_tiled(Geo g, Ws w) {
   extern __shared__ __align__(16) float dsm[];
   constexpr int R = kTileRows;
   const int N = g.N;
@@ -280,75 +282,76 @@ __global__ void __launch_bounds__(kDraftThreads, 1) k_draft_tiled(Geo g, Ws w) {
   }
   const float* kavg = w.kavg + (size_t)bh * N * D;
   const float* kmax = w.kmax + (size_t)bh * N * D;
-  unsigned long long acc[2][2][R / 2];            // [key][map][row pair]
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int m = 0; m < 2; ++m)
-#pragma unroll
-      for (int p = 0; p < R / 2; ++p) acc[i][m][p] = 0ull;
   __syncthreads();                                // the transposed query rows are in place
   // this thread's two key blocks (a lane past the last block recomputes the last one);
-  // threads t >= KL only rank
+  // threads t >= KL only rank. One map at a time: 2 keys x 8 row pairs of accumulators.
   const int ja = tid < N ? tid : N - 1, jb = tid + KL < N ? tid + KL : N - 1;
-  if (tid < KL) {
-  const float4* ka[2] = {reinterpret_cast<const float4*>(kavg + (size_t)ja * D),
-                         reinterpret_cast<const float4*>(kavg + (size_t)jb * D)};
-  const float4* km[2] = {reinterpret_cast<const float4*>(kmax + (size_t)ja * D),
-                         reinterpret_cast<const float4*>(kmax + (size_t)jb * D)};
-#pragma unroll 1
-  for (int c4 = 0; c4 < D / 4; ++c4) {
-    float4 kv[2][2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      kv[i][0] = __ldg(ka[i] + c4);
-      kv[i][1] = __ldg(km[i] + c4);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const float4* qp = reinterpret_cast<const float4*>(qT + (m * D + 4 * c4 + e) * R);
-        unsigned long long qq[R / 2];
-#pragma unroll
-        for (int f = 0; f < R / 4; ++f) {
-          const float4 x = qp[f];
-          qq[2 * f] = pk2f(x.x, x.y);
-          qq[2 * f + 1] = pk2f(x.z, x.w);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const float k1 = e == 0 ? kv[i][m].x : (e == 1 ? kv[i][m].y : (e == 2 ? kv[i][m].z : kv[i][m].w));
-          const unsigned long long kk = pk2f(k1, k1);
-#pragma unroll
-          for (int p = 0; p < R / 2; ++p) acc[i][m][p] = fma2f(qq[p], kk, acc[i][m][p]);
-        }
-      }
-    }
-  }
   const bool mass = !(g.flags & DA2_FLAG_NO_MASS_CORRECTION);
   const int fpf = g.ny * g.nx;
+  float lc[2] = {0.0f, 0.0f};
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int j = tid + i * KL;
-    if (j >= N) continue;
-    float lc = 0.0f;
-    if (mass) {
+    if (mass && j < N) {
       const int rem = j % fpf, by = rem / g.nx, bx = rem - by * g.nx;
       const int hv = min(g.ph, g.Hf - by * g.ph), wv = min(g.pw, g.Wf - bx * g.pw);
-      lc = logf((float)(hv * wv));
-    }
-#pragma unroll
-    for (int p = 0; p < R / 2; ++p) {
-      float a0, a1, m0, m1;
-      upk2f(acc[i][0][p], a0, a1);
-      upk2f(acc[i][1][p], m0, m1);
-      la[(2 * p) * N + j] = fmaf(g.sm_scale, a0, lc);
-      la[(2 * p + 1) * N + j] = fmaf(g.sm_scale, a1, lc);
-      lm[(2 * p) * N + j] = fmaf(g.sm_scale, m0, lc);
-      lm[(2 * p + 1) * N + j] = fmaf(g.sm_scale, m1, lc);
+      lc[i] = logf((float)(hv * wv));
     }
   }
+  if (tid < KL) {
+#pragma unroll 1
+    for (int m = 0; m < 2; ++m) {
+      const float* kb = m == 0 ? kavg : kmax;
+      const float4* kp[2] = {reinterpret_cast<const float4*>(kb + (size_t)ja * D),
+                             reinterpret_cast<const float4*>(kb + (size_t)jb * D)};
+      const float* qm = qT + m * D * R;
+      unsigned long long acc[2][R / 2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int p = 0; p < R / 2; ++p) acc[i][p] = 0ull;
+      // acc += q[c] k[c] over the channels of one float4 of each key, c ascending
+      auto step = [&](int c4, const float4 (&kv)[2]) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4* qp = reinterpret_cast<const float4*>(qm + (4 * c4 + e) * R);
+          unsigned long long kk[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float k1 = e == 0 ? kv[i].x : (e == 1 ? kv[i].y : (e == 2 ? kv[i].z : kv[i].w));
+            kk[i] = pk2f(k1, k1);
+          }
+#pragma unroll
+          for (int f = 0; f < R / 4; ++f) {
+            const float4 x = qp[f];
+            const unsigned long long q0 = pk2f(x.x, x.y), q1 = pk2f(x.z, x.w);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              acc[i][2 * f] = fma2f(q0, kk[i], acc[i][2 * f]);
+              acc[i][2 * f + 1] = fma2f(q1, kk[i], acc[i][2 * f + 1]);
+            }
+          }
+        }
+      };
+#pragma unroll 2
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 kv[2] = {__ldg(kp[0] + c4), __ldg(kp[1] + c4)};
+        step(c4, kv);
+      }
+      float* lo = m == 0 ? la : lm;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int j = tid + i * KL;
+        if (j >= N) continue;
+#pragma unroll
+        for (int p = 0; p < R / 2; ++p) {
+          float a0, a1;
+          upk2f(acc[i][p], a0, a1);
+          lo[(2 * p) * N + j] = fmaf(g.sm_scale, a0, lc[i]);
+          lo[(2 * p + 1) * N + j] = fmaf(g.sm_scale, a1, lc[i]);
+        }
+      }
+    }
   }
   __syncthreads();
   rank_rows(g, w, la, lm, hist, bh, i0, rows, warp, lane, blockDim.x / 32);
@@ -378,9 +381,13 @@ cudaError_t launch_draft_select(const Geo& g, const Ws& w, cudaStream_t st) {
     if (g.d == 128) {
       e = cudaFuncSetAttribute(k_draft_tiled<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(k_draft_tiled<128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return e;
       k_draft_tiled<128><<<grid, KL, smem, st>>>(g, w);
     } else {
       e = cudaFuncSetAttribute(k_draft_tiled<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(k_draft_tiled<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
       if (e != cudaSuccess) return e;
       k_draft_tiled<64><<<grid, KL, smem, st>>>(g, w);
     }
