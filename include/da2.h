@@ -88,6 +88,12 @@ enum {
      place, results identical. da2_forward_host then runs unpipelined. (The pages fix no
      tensor layout.) */
   DA2_FLAG_LAYOUT_BTHD = 4,
+  /* Debug aid: every workspace region is followed by a 256-byte guard (the workspace grows
+     accordingly; da2_workspace_size and da2_workspace_views account for it). da2_prepare
+     fills the guards with 0xA5 bytes and every stage call checks them after its kernels: a
+     changed guard byte sets bit 4 of the workspace error word (DA2_ERR_TIMEOUT from
+     da2_get_error). Costs two small launches per stage; off in normal use. */
+  DA2_FLAG_DEBUG_CANARY = 8,
   /* Test hook for the failure path, never needed in use: da2_attention's copy engine
      withholds its first K/V tile, so a bounded device wait must run out. Every bounded
      wait's limit drops from 2 s to 50 ms; the launch sets the workspace error word, stops
@@ -104,7 +110,8 @@ typedef enum da2_status {
   DA2_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
   DA2_ERR_WORKSPACE = 4,    /* ws_bytes smaller than da2_workspace_size */
   DA2_ERR_CUDA = 5,         /* a CUDA call or launch failed */
-  DA2_ERR_TIMEOUT = 6,      /* a kernel's bounded wait ran out (device error word set) */
+  DA2_ERR_TIMEOUT = 6,      /* the device error word is set (a bounded wait ran out, a bad
+                               index, or an overwritten guard region) */
   DA2_ERR_SCRATCH_TOO_SMALL = 7 /* da2_forward_noalloc: the configuration's workspace does
                                    not fit the library's built-in 64 MiB device scratch */
 } da2_status;
@@ -138,7 +145,14 @@ typedef enum da2_status {
               max(n8,1), n4s = max(n4max,1), nms = max(nm,1)); with the adaptive budget a
               row's FP4 list holds its n4 .. n4max blocks followed by -1 entries.
      scores   fp32 [BH][N][N] (only with DA2_FLAG_EXPORT_SCORES, else size 0).
-     err      u32 device error word (0 = no error). */
+     err      u32 device error word (0 = no error): bit 1 a bounded wait ran out, bit 2 an
+              index or count of the selection was out of range, bit 4 a guard region of
+              DA2_FLAG_DEBUG_CANARY was overwritten.
+   With DA2_FLAG_DEBUG_CANARY a 256-byte guard follows every region above.
+   A DA2_DEBUG build of the library (libda2_debug.so) also checks the selection's lists
+   and tags before the attention (indices in range and ascending, tags of the right class,
+   counts equal to the budgets) and makes every stage call wait for its stream and return
+   DA2_ERR_TIMEOUT at once when the error word is set. */
 typedef struct da2_views {
   int N, bs, T, Tp, ny, nx, n8, n4, kv4;
   size_t tile8_qk, tile4_qk, tile8_v, tile4_v, sf_qk, sf_v;
@@ -173,6 +187,17 @@ da2_status da2_draft_select(const da2_config* cfg, void* ws, size_t ws_bytes,
    set the workspace error word (read it with da2_get_error). Asynchronous. */
 da2_status da2_attention(const da2_config* cfg, void* ws, size_t ws_bytes, void* out,
                          cudaStream_t stream);
+
+/* Debug aid (no counterpart in the paper): checks the output contract of
+   da2_draft_select on a selected workspace before it reaches the attention. Per (b, h,
+   query block) the FP8, mixed and FP4 lists must hold in-range, strictly ascending KV
+   blocks tagged 2, 3 and 1, the FP4 list may end in -1 padding only after its last block,
+   and the row must hold exactly n8 FP8 and nm mixed tags and n4..n4max FP4 tags. A
+   violation sets bit 2 of the workspace error word (read it with da2_get_error). Reads
+   only the workspace; asynchronous on `stream`. DA2_DEBUG builds run it inside
+   da2_draft_select. */
+da2_status da2_check_selection(const da2_config* cfg, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
 
 /* da2_prepare, da2_draft_select and da2_attention in order on one stream. */
 da2_status da2_forward(const da2_config* cfg, const void* q, const void* k, const void* v,

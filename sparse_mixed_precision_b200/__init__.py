@@ -24,10 +24,12 @@ import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libda2.so")
+LIB_DEBUG_PATH = os.path.join(_HERE, "libda2_debug.so")   # DA2_DEBUG build (see use_library)
 
 FLAG_EXPORT_SCORES = 1
 FLAG_NO_MASS_CORRECTION = 2
 FLAG_LAYOUT_BTHD = 4          # q, k, v, out token-major [B, T, H, d]
+FLAG_DEBUG_CANARY = 8         # guard region after every workspace region, checked per stage
 FLAG_TEST_STALL = 256         # test hook: a bounded wait of the attention kernel runs out
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned pointer",
@@ -66,12 +68,23 @@ class DA2Error(RuntimeError):
 _lib = None
 
 
+def use_library(path: str) -> str:
+    """Selects the build of the library that the binding calls from the next call on (for
+    example LIB_DEBUG_PATH, built by `python -m sparse_mixed_precision_b200.build --debug`);
+    returns the previous path."""
+    global LIB_PATH, _lib
+    prev, LIB_PATH, _lib = LIB_PATH, path, None
+    return prev
+
+
 def lib():
-    """The loaded libda2.so; raises if it has not been built."""
+    """The loaded library (libda2.so unless use_library chose another build); raises if it
+    has not been built."""
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"libda2.so not built ({LIB_PATH}); run sparse_mixed_precision_b200.build")
+            raise RuntimeError(f"{os.path.basename(LIB_PATH)} not built ({LIB_PATH}); "
+                               "run sparse_mixed_precision_b200.build")
         L = ctypes.CDLL(LIB_PATH)
         vp, sz, cp = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Config)
         sigs = {
@@ -84,6 +97,7 @@ def lib():
             "da2_forward_host": [cp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "da2_get_error": [vp, sz, cp, vp, ctypes.POINTER(ctypes.c_uint32)],
             "da2_forward_noalloc": [cp, vp, vp, vp, vp, vp],
+            "da2_check_selection": [cp, vp, sz, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -100,7 +114,8 @@ def lib():
 
 EXPORTED = ("da2_workspace_size", "da2_workspace_views", "da2_prepare", "da2_draft_select",
             "da2_attention", "da2_forward", "da2_forward_host", "da2_get_error",
-            "da2_status_string", "da2_forward_noalloc", "da2_last_cuda_error")
+            "da2_status_string", "da2_forward_noalloc", "da2_last_cuda_error",
+            "da2_check_selection")
 
 
 def config(w, flags: int = 0, sm_scale: float = 0.0) -> Config:
@@ -145,6 +160,13 @@ def prepare(cfg, q, k, v, ws, stream=None):
 def draft_select(cfg, ws, stream=None):
     _check("da2_draft_select", lib().da2_draft_select(ctypes.byref(cfg), _ptr(ws), ws.numel(),
                                                       _stream(stream)))
+
+
+def check_selection(cfg, ws, stream=None):
+    """Debug aid: checks the selection's lists and tags in ws (da2_check_selection); a
+    violation shows up in get_error."""
+    _check("da2_check_selection", lib().da2_check_selection(ctypes.byref(cfg), _ptr(ws), ws.numel(),
+                                                            _stream(stream)))
 
 
 def attention(cfg, ws, out, stream=None):

@@ -2,6 +2,9 @@
 #include <cmath>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
+#include "checks.cuh"
 #include "common.cuh"
 
 namespace da2 {
@@ -34,7 +37,7 @@ da2_status check_config(const da2_config* c) {
       (c->pct_fp4_max < c->pct_fp4 || c->pct_fp8 + c->pct_mix + c->pct_fp4_max > 100))
     return DA2_ERR_INVALID_ARG;
   if (c->flags & ~(DA2_FLAG_EXPORT_SCORES | DA2_FLAG_NO_MASS_CORRECTION | DA2_FLAG_LAYOUT_BTHD |
-                   DA2_FLAG_TEST_STALL))
+                   DA2_FLAG_DEBUG_CANARY | DA2_FLAG_TEST_STALL))
     return DA2_ERR_INVALID_ARG;
   if (c->d != 64 && c->d != 128) return DA2_ERR_UNSUPPORTED;
   const long bs = (long)c->ph * c->pw;
@@ -46,8 +49,12 @@ da2_status check_config(const da2_config* c) {
   return DA2_OK;
 }
 
-void fill_views(const da2_config* c, da2_views* v) {
+// With DA2_FLAG_DEBUG_CANARY every region is followed by a guard of kGuardBytes (its offset
+// recorded in *gl when given).
+void fill_views(const da2_config* c, da2_views* v, GuardList* gl = nullptr) {
   std::memset(v, 0, sizeof(*v));
+  const bool guards = (c->flags & DA2_FLAG_DEBUG_CANARY) != 0;
+  if (gl) gl->n = 0;
   v->ny = (c->Hf + c->ph - 1) / c->ph;
   v->nx = (c->Wf + c->pw - 1) / c->pw;
   v->N = c->F * v->ny * v->nx;
@@ -73,7 +80,15 @@ void fill_views(const da2_config* c, da2_views* v) {
   v->sf_v = (v->kv4 / 64) * 512;
   const size_t n8s = v->n8 > 0 ? v->n8 : 1, n4s = v->n4max > 0 ? v->n4max : 1, nms = v->nm > 0 ? v->nm : 1;
   size_t off = 0;
-  auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + bytes); return o; };
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    if (guards) {
+      if (gl && gl->n < kMaxGuards) gl->off[gl->n++] = off;
+      off += kGuardBytes;
+    }
+    return o;
+  };
   v->q8 = take(BH * N * v->tile8_qk);
   v->k8 = take(BH * N * v->tile8_qk);
   v->v8 = take(BH * N * v->tile8_v);
@@ -144,12 +159,13 @@ Ws make_ws(void* base, const da2_views& v) {
 }
 
 // Common checks for the stage calls; fills views / geo / ws on success.
-da2_status setup(const da2_config* cfg, void* ws, size_t ws_bytes, da2_views* v, Geo* g, Ws* w) {
+da2_status setup(const da2_config* cfg, void* ws, size_t ws_bytes, da2_views* v, Geo* g, Ws* w,
+                 GuardList* gl = nullptr) {
   da2_status s = check_config(cfg);
   if (s != DA2_OK) return s;
   if (!ws) return DA2_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DA2_ERR_ALIGNMENT;
-  fill_views(cfg, v);
+  fill_views(cfg, v, gl);
   if (ws_bytes < v->total) return DA2_ERR_WORKSPACE;
   *g = make_geo(cfg, *v);
   *w = make_ws(ws, *v);
@@ -164,6 +180,30 @@ da2_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return DA2_OK;
   g_last_cuda = e;
   return DA2_ERR_CUDA;
+}
+
+// An NVTX range around one library call (visible in a profiler's timeline; no cost without
+// an attached tool).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
+// End of a stage call: with DA2_FLAG_DEBUG_CANARY the guard regions are checked (a change
+// sets kErrCanary in the error word); a DA2_DEBUG build then waits for the stream and
+// returns DA2_ERR_TIMEOUT at once if the error word is set (the word stays set for
+// da2_get_error).
+da2_status finish_stage(const da2_config* cfg, const Ws& w, void* ws, const GuardList& gl,
+                        cudaError_t e, cudaStream_t stream) {
+  if (e == cudaSuccess && (cfg->flags & DA2_FLAG_DEBUG_CANARY))
+    e = launch_guards(static_cast<uint8_t*>(ws), gl, true, w.err, stream);
+#ifdef DA2_DEBUG
+  uint32_t h = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&h, w.err, 4, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess && h != 0) return DA2_ERR_TIMEOUT;
+#endif
+  return cuda_status(e);
 }
 
 }  // namespace
@@ -190,33 +230,52 @@ da2_status da2_workspace_views(const da2_config* cfg, da2_views* views) {
 
 da2_status da2_prepare(const da2_config* cfg, const void* q, const void* k, const void* v,
                        void* ws, size_t ws_bytes, cudaStream_t stream) {
-  da2_views vw; Geo g; Ws w;
-  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
+  const NvtxRange range("da2_prepare");
+  da2_views vw; Geo g; Ws w; GuardList gl;
+  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w, &gl);
   if (s != DA2_OK) return s;
   if (!q || !k || !v) return DA2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return DA2_ERR_ALIGNMENT;
-  return cuda_status(launch_prepare(g, w, q, k, v, stream));
+  cudaError_t e = cudaSuccess;
+  if (cfg->flags & DA2_FLAG_DEBUG_CANARY) e = launch_guards(static_cast<uint8_t*>(ws), gl, false, w.err, stream);
+  if (e == cudaSuccess) e = launch_prepare(g, w, q, k, v, stream);
+  return finish_stage(cfg, w, ws, gl, e, stream);
 }
 
 da2_status da2_draft_select(const da2_config* cfg, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  da2_views vw; Geo g; Ws w;
-  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
+  const NvtxRange range("da2_draft_select");
+  da2_views vw; Geo g; Ws w; GuardList gl;
+  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w, &gl);
   if (s != DA2_OK) return s;
-  return cuda_status(launch_draft_select(g, w, stream));
+  cudaError_t e = launch_draft_select(g, w, stream);
+#ifdef DA2_DEBUG
+  if (e == cudaSuccess) e = launch_check_lists(g, w, stream);
+#endif
+  return finish_stage(cfg, w, ws, gl, e, stream);
 }
 
 da2_status da2_attention(const da2_config* cfg, void* ws, size_t ws_bytes, void* out,
                          cudaStream_t stream) {
-  da2_views vw; Geo g; Ws w;
-  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
+  const NvtxRange range("da2_attention");
+  da2_views vw; Geo g; Ws w; GuardList gl;
+  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w, &gl);
   if (s != DA2_OK) return s;
   if (!out) return DA2_ERR_INVALID_ARG;
   if (!aligned16(out)) return DA2_ERR_ALIGNMENT;
-  return cuda_status(launch_attention_tc(g, w, out, stream));
+  return finish_stage(cfg, w, ws, gl, launch_attention_tc(g, w, out, stream), stream);
+}
+
+da2_status da2_check_selection(const da2_config* cfg, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const NvtxRange range("da2_check_selection");
+  da2_views vw; Geo g; Ws w;
+  const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w);
+  if (s != DA2_OK) return s;
+  return cuda_status(launch_check_lists(g, w, stream));
 }
 
 da2_status da2_forward(const da2_config* cfg, const void* q, const void* k, const void* v,
                        void* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const NvtxRange range("da2_forward");
   da2_status s = da2_prepare(cfg, q, k, v, ws, ws_bytes, stream);
   if (s != DA2_OK) return s;
   s = da2_draft_select(cfg, ws, ws_bytes, stream);
@@ -253,6 +312,7 @@ constexpr int kHostGroups = 16;   // head groups the host-buffer path pipelines 
 da2_status da2_forward_host(const da2_config* cfg, const void* q_host, const void* k_host,
                             const void* v_host, void* out_host, void* dq, void* dk, void* dv,
                             void* dout, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const NvtxRange range("da2_forward_host");
   const da2_status s0 = check_config(cfg);
   if (s0 != DA2_OK) return s0;
   if (!q_host || !k_host || !v_host || !out_host || !dq || !dk || !dv || !dout)

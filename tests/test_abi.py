@@ -85,7 +85,7 @@ def test_flags_checked_and_layout_flag_keeps_the_workspace():
     L = da2.lib()
     n = ctypes.c_size_t()
     w = WORKLOADS["tiny"]
-    assert L.da2_workspace_size(ctypes.byref(da2.config(w, flags=8)), ctypes.byref(n)) == 1
+    assert L.da2_workspace_size(ctypes.byref(da2.config(w, flags=16)), ctypes.byref(n)) == 1
     # the token-major layout changes where q/k/v/out live, not the workspace
     assert da2.workspace_views(da2.config(w, flags=da2.FLAG_LAYOUT_BTHD)) == da2.workspace_views(da2.config(w))
 
@@ -109,7 +109,7 @@ def test_noalloc_host_side_refusals():
     L = da2.lib()
     p = ctypes.c_void_p(0x100000)
     assert L.da2_forward_noalloc(None, p, p, p, p, None) == 1
-    bad = da2.config(WORKLOADS["tiny"], flags=8)
+    bad = da2.config(WORKLOADS["tiny"], flags=16)
     assert L.da2_forward_noalloc(ctypes.byref(bad), p, p, p, p, None) == 1
     assert L.da2_forward_noalloc(ctypes.byref(da2.config(scaled(WORKLOADS["tiny"], d=96))),
                                  p, p, p, p, None) == 2
@@ -157,3 +157,52 @@ def test_adaptive_budget_views_and_limits():
                 dict(pct_fp4_max=50, adapt_tau=-1.0), dict(pct_fp4_max=50, adapt_tau=float("inf"))):
         cfg = da2.config(scaled(WORKLOADS["tiny"], **bad))
         assert L.da2_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 1, bad
+
+
+REGIONS = ("q8", "k8", "v8", "q4", "k4", "v4", "sfq4", "sfk4", "sfv4", "sq", "sk", "sv", "vamax",
+           "qavg", "qmax", "kavg", "kmax", "tags", "list8", "list4", "listm", "err")
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan720", "hunyuan720"])
+def test_canary_layout_puts_a_guard_after_every_region(name):
+    """DA2_FLAG_DEBUG_CANARY: every region keeps its size and is followed by at least 256
+    bytes that no region uses; the workspace grows by one guard per region."""
+    w = WORKLOADS[name]
+    plain = da2.workspace_views(da2.config(w))
+    guarded = da2.workspace_views(da2.config(w, flags=da2.FLAG_DEBUG_CANARY))
+    for k in ("N", "bs", "n8", "n4", "n4max", "nm", "tile8_qk", "tile4_qk", "tile8_v", "tile4_v"):
+        assert guarded[k] == plain[k], k
+
+    def spans(v):
+        order = sorted(REGIONS, key=lambda r: v[r])
+        nxt = {r: (v[order[i + 1]] if i + 1 < len(order) else v["total"]) for i, r in enumerate(order)}
+        return order, nxt
+
+    order_p, next_p = spans(plain)
+    order_g, next_g = spans(guarded)
+    assert order_p == order_g
+    for r in order_g:
+        # the region's bytes in the plain layout (up to its 256-byte rounding) are followed
+        # by a guard of at least 256 bytes in the guarded layout
+        size = next_p[r] - plain[r]
+        assert next_g[r] - guarded[r] >= size + 256, r
+    assert guarded["total"] >= plain["total"] + 256 * len(REGIONS)
+
+
+def test_debug_library_exports_every_declared_symbol():
+    """The DA2_DEBUG build (built by __graft_entry__.build) exports the same C ABI."""
+    if not os.path.exists(da2.LIB_DEBUG_PATH):
+        pytest.skip("libda2_debug.so not built")
+    L = ctypes.CDLL(da2.LIB_DEBUG_PATH)
+    for n in sorted(declared_symbols()):
+        assert hasattr(L, n), n
+
+
+def test_check_selection_rejects_bad_arguments_without_touching_the_device():
+    L = da2.lib()
+    cfg = da2.config(WORKLOADS["tiny"])
+    n = da2.workspace_size(cfg)
+    assert L.da2_check_selection(None, ctypes.c_void_p(0x100000), n, None) == 1
+    assert L.da2_check_selection(ctypes.byref(cfg), None, n, None) == 1
+    assert L.da2_check_selection(ctypes.byref(cfg), ctypes.c_void_p(0x1008), n, None) == 3
+    assert L.da2_check_selection(ctypes.byref(cfg), ctypes.c_void_p(0x100000), n - 1, None) == 4
