@@ -145,6 +145,9 @@ typedef enum da2_status {
               max(n8,1), n4s = max(n4max,1), nms = max(nm,1)); with the adaptive budget a
               row's FP4 list holds its n4 .. n4max blocks followed by -1 entries.
      scores   fp32 [BH][N][N] (only with DA2_FLAG_EXPORT_SCORES, else size 0).
+     dlog     fp32 [BH][N][2][np] the two draft logit rows (average map, max map) of every
+              query block, written and read by da2_draft_select (scratch; size 0 when
+              N > 1024).
      err      u32 device error word (0 = no error): bit 1 a bounded wait ran out, bit 2 an
               index or count of the selection was out of range, bit 4 a guard region of
               DA2_FLAG_DEBUG_CANARY was overwritten.
@@ -162,6 +165,8 @@ typedef struct da2_views {
   int nm;               /* mixed KV blocks per query block */
   size_t listm;
   int n4max;            /* FP4 list length (n4 unless the adaptive budget is on) */
+  size_t dlog;          /* draft logits scratch (N <= 1024), see below */
+  int np;               /* its row length: N rounded up to a multiple of 4 */
 } da2_views;
 
 /* Workspace bytes needed for `cfg` (host only, no CUDA call). */

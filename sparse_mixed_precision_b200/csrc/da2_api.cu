@@ -10,7 +10,7 @@
 namespace da2 {
 cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
                            const void* v, cudaStream_t st);
-cudaError_t launch_draft_select(const Geo& g, const Ws& w, cudaStream_t st);
+cudaError_t launch_draft_select(const Geo& g, const Ws& w, float* dlog, int np, cudaStream_t st);
 cudaError_t launch_attention_tc(const Geo& g, const Ws& w, void* out, cudaStream_t st);
 da2_status noalloc_scratch(void** ptr, size_t* bytes);   // da2_noalloc.cu
 }  // namespace da2
@@ -111,6 +111,8 @@ void fill_views(const da2_config* c, da2_views* v, GuardList* gl = nullptr) {
   v->list4 = take(BH * N * n4s * 2);
   v->listm = take(BH * N * nms * 2);
   v->scores = take((c->flags & DA2_FLAG_EXPORT_SCORES) ? BH * N * N * 4 : 0);
+  v->np = (int)((N + 3) / 4 * 4);
+  v->dlog = take(N <= 1024 ? BH * N * 2 * (size_t)v->np * 4 : 0);
   v->err = take(4);
   v->total = off;
 }
@@ -247,7 +249,8 @@ da2_status da2_draft_select(const da2_config* cfg, void* ws, size_t ws_bytes, cu
   da2_views vw; Geo g; Ws w; GuardList gl;
   const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w, &gl);
   if (s != DA2_OK) return s;
-  cudaError_t e = launch_draft_select(g, w, stream);
+  float* dlog = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + vw.dlog);
+  cudaError_t e = launch_draft_select(g, w, dlog, vw.np, stream);
 #ifdef DA2_DEBUG
   if (e == cudaSuccess) e = launch_check_lists(g, w, stream);
 #endif

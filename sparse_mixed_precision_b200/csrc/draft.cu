@@ -8,12 +8,14 @@
 // Low-Resolution Attention Guidance", Abstract: the draft map is the attention of the
 // pooled queries over the pooled keys.
 //
-// One CTA takes R query blocks of one (b, h): it forms both draft logit rows against all N
-// key blocks (fp32 FMA), turns each into a row softmax, averages the two maps into the
-// score, and each warp ranks its rows with an exact radix select over the score bits
-// (ties broken by the lower block index), then writes tags and the ascending index lists of
-// the kept classes (FP8, mixed, FP4).
+// Up to 1024 key blocks: the two logit maps of every (b, h) run on the tensor cores into a
+// scratch (k_draft_logits_tc), then k_draft_rank turns each query block's two rows into row
+// softmaxes, averages them into the score, and ranks the row with an exact radix select
+// over the score bits (ties broken by the lower block index), writing tags and the
+// ascending index lists of the kept classes (FP8, mixed, FP4). Above 1024 key blocks one
+// kernel (k_draft_select) forms the logits with fp32 FMAs and ranks in the same way.
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace da2 {
 
@@ -233,132 +235,245 @@ __global__ void __launch_bounds__(kDraftThreads) k_draft_select(Geo g, Ws w, int
   rank_rows(g, w, la, lm, hist, bh, i0, rows, warp, lane, kDraftWarps);
 }
 
-// Register-tiled draft logits for up to 1024 key blocks: a CTA of KL = blockDim.x threads
-// takes 16 query blocks of one (b, h); thread t owns key blocks t and t + KL and all 16 query
-// rows, one map after the other, as packed pairs of rows (f32x2 FMA). The pooled queries sit
-// in shared memory transposed ([map][channel][row], read as float4 by every thread alike);
-// each thread streams its own two pooled key rows (16-byte loads through L1). Then the same
-// per-row ranking as the general kernel. At 64 registers a thread and about 111 KB of
-// shared memory (up to 630 key blocks) two CTAs share an SM, so that the latency of one
-// CTA's phases is hidden by the other's warps.
-constexpr int kTileRows = 16;
+// ---- draft logits on the tensor cores (N <= 1024) ----
+// The two draft maps are dense contractions per head, L_map = Q_map K_map^T ([N, d] x [d, N]).
+// They run as tcgen05 MMAs of kind::tf32. A tf32 operand keeps 10 of fp32's 23 mantissa
+// bits, so each operand x is split into hi = x with its low 13 mantissa bits cleared (exact
+// in tf32) and lo = x - hi (exact in fp32, 13 significant bits of which tf32 keeps 10), and
+// each K step accumulates hi_a hi_b + hi_a lo_b + lo_a hi_b in fp32: every product of tf32
+// significands is exact, the dropped lo_a lo_b and lo's truncation are below 2^-20 of |a b|.
+// One CTA takes 128 query blocks (TMEM lanes) of one (b, h) and a range of 128-key tiles,
+// one map after the other: the queries of the map (both parts, K-major core-matrix layout,
+// all d channels) stay in shared memory, the keys stream in 32-channel stages (double
+// buffered), the accumulator of a tile sits in one of two 128-column TMEM buffers while the
+// other one is read out. The logits (sm_scale * acc + ln c_j) go to a global scratch of
+// [B*H][N][2][NP] fp32 rows that the ranking kernel reads.
+constexpr int kTcRows = 128, kTcKeys = 128, kTcKC = 32, kTcThreads = 256;
 
-__device__ __forceinline__ unsigned long long pk2f(float lo, float hi) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+  // D fp32, A and B tf32, both K-major, N / 8, M / 16
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-__device__ __forceinline__ void upk2f(unsigned long long v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
-__device__ __forceinline__ unsigned long long fma2f(unsigned long long a, unsigned long long b,
-                                                    unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ unsigned long long draft_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait on an mbarrier phase; a wait that runs out sets the error word and returns.
+__device__ __forceinline__ void draft_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                           unsigned long long limit_ns) {
+  if (tc::mbar_try_wait(bar, parity)) return;
+  const unsigned long long t0 = draft_ns();
+  while (!tc::mbar_try_wait(bar, parity)) {
+    if (draft_ns() - t0 > limit_ns) {
+      set_error(err, kErrWaitTimeout);
+      return;
+    }
+  }
+}
+// tf32 high part (low 13 mantissa bits cleared) and the exact remainder.
+__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
+  hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+  lo = x - hi;
+}
+// 8 rows x 4 float4 of a row-major fp32 [rows][D] source into the hi and lo tiles (K-major
+// core matrices: rows of `rowbytes` bytes); lane l takes row r0 + (l & 7), float4 c0 + (l >> 3),
+// so a warp reads 8 x 64 contiguous bytes and writes 512 contiguous bytes of each tile.
+__device__ __forceinline__ void stage_split(const float* src, int ld, int r0, int rvalid, int c0,
+                                            uint8_t* hi, uint8_t* lo, uint32_t rowbytes, int lane) {
+  const int r = r0 + (lane & 7), c4 = c0 + (lane >> 3);
+  float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (r < rvalid) x = __ldg(reinterpret_cast<const float4*>(src + (size_t)r * ld) + c4);
+  float4 h, l;
+  split_tf32(x.x, h.x, l.x);
+  split_tf32(x.y, h.y, l.y);
+  split_tf32(x.z, h.z, l.z);
+  split_tf32(x.w, h.w, l.w);
+  const uint32_t off = kmajor_off((uint32_t)r, (uint32_t)c4 * 16u, rowbytes);
+  *reinterpret_cast<float4*>(hi + off) = h;
+  *reinterpret_cast<float4*>(lo + off) = l;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kDraftThreads, 2) k_draft_tiled(Geo g, Ws w) {
-  extern __shared__ __align__(16) float dsm[];
-  constexpr int R = kTileRows;
-  const int N = g.N;
-  const int KL = ((N + 1) / 2 + 31) / 32 * 32;    // key lanes: keys t and t + KL (t < KL)
-  float* qT = dsm;                                // [2][D][R]
-  float* la = qT + 2 * D * R;                     // [R][N]
-  float* lm = la + R * N;                         // [R][N]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(lm + R * N);   // [warps][256]
-  const int bh = blockIdx.y, i0 = blockIdx.x * R;
-  const int rows = min(R, N - i0);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  const float* qavg = w.qavg + ((size_t)bh * N + i0) * D;
-  const float* qmax = w.qmax + ((size_t)bh * N + i0) * D;
-  for (int u = tid; u < R * D; u += blockDim.x) {
-    const int r = u / D, c = u - r * D;
-    const bool ok = r < rows;
-    qT[c * R + r] = ok ? __ldg(qavg + u) : 0.0f;
-    qT[(D + c) * R + r] = ok ? __ldg(qmax + u) : 0.0f;
+__global__ void __launch_bounds__(kTcThreads, 1) k_draft_logits_tc(Geo g, Ws w, float* dlog, int NP, int tiles_per_cta) {
+  constexpr uint32_t A_PART = kTcRows * D * 4;          // one part of the queries, all channels
+  constexpr uint32_t B_PART = kTcKeys * kTcKC * 4;      // one part of a key stage
+  constexpr int NKC = D / kTcKC;                        // key stages per tile
+  extern __shared__ __align__(1024) uint8_t dsm_tc[];
+  uint8_t* a_hi = dsm_tc;
+  uint8_t* a_lo = dsm_tc + A_PART;
+  uint8_t* b_st = dsm_tc + 2 * A_PART;                  // [stage][part][B_PART]
+  float* lcs = reinterpret_cast<float*>(b_st + 4 * B_PART);          // ln c_j, [1024]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(lcs + 1024);           // stage_free[2], acc_full[2]
+  __shared__ uint32_t tmem_holder;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int N = g.N, bh = blockIdx.y, i0 = blockIdx.x * kTcRows;
+  const int NT = (N + kTcKeys - 1) / kTcKeys;
+  const int t0 = blockIdx.z * tiles_per_cta, t1 = min(NT, t0 + tiles_per_cta);
+  if (t0 >= t1) return;
+  const int nt = t1 - t0;
+  if (warp == 0) {
+    tc::tmem_alloc(&tmem_holder, 2 * kTcKeys);
+    tc::tmem_relinquish();
   }
-  const float* kavg = w.kavg + (size_t)bh * N * D;
-  const float* kmax = w.kmax + (size_t)bh * N * D;
-  __syncthreads();                                // the transposed query rows are in place
-  // this thread's two key blocks (a lane past the last block recomputes the last one);
-  // threads t >= KL only rank. One map at a time: 2 keys x 8 row pairs of accumulators.
-  const int ja = tid < N ? tid : N - 1, jb = tid + KL < N ? tid + KL : N - 1;
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
+    tc::fence_mbar_init();
+  }
   const bool mass = !(g.flags & DA2_FLAG_NO_MASS_CORRECTION);
   const int fpf = g.ny * g.nx;
-  float lc[2] = {0.0f, 0.0f};
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int j = tid + i * KL;
-    if (mass && j < N) {
+  for (int j = tid; j < N; j += kTcThreads) {
+    float lc = 0.0f;
+    if (mass) {
       const int rem = j % fpf, by = rem / g.nx, bx = rem - by * g.nx;
       const int hv = min(g.ph, g.Hf - by * g.ph), wv = min(g.pw, g.Wf - bx * g.pw);
-      lc[i] = logf((float)(hv * wv));
+      lc = logf((float)(hv * wv));
     }
+    lcs[j] = lc;
   }
-  if (tid < KL) {
-#pragma unroll 1
-    for (int m = 0; m < 2; ++m) {
-      const float* kb = m == 0 ? kavg : kmax;
-      const float4* kp[2] = {reinterpret_cast<const float4*>(kb + (size_t)ja * D),
-                             reinterpret_cast<const float4*>(kb + (size_t)jb * D)};
-      const float* qm = qT + m * D * R;
-      unsigned long long acc[2][R / 2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int p = 0; p < R / 2; ++p) acc[i][p] = 0ull;
-      // acc += q[c] k[c] over the channels of one float4 of each key, c ascending
-      auto step = [&](int c4, const float4 (&kv)[2]) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4* qp = reinterpret_cast<const float4*>(qm + (4 * c4 + e) * R);
-          unsigned long long kk[2];
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const float k1 = e == 0 ? kv[i].x : (e == 1 ? kv[i].y : (e == 2 ? kv[i].z : kv[i].w));
-            kk[i] = pk2f(k1, k1);
-          }
-#pragma unroll
-          for (int f = 0; f < R / 4; ++f) {
-            const float4 x = qp[f];
-            const unsigned long long q0 = pk2f(x.x, x.y), q1 = pk2f(x.z, x.w);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              acc[i][2 * f] = fma2f(q0, kk[i], acc[i][2 * f]);
-              acc[i][2 * f + 1] = fma2f(q1, kk[i], acc[i][2 * f + 1]);
-            }
-          }
-        }
-      };
-#pragma unroll 2
-      for (int c4 = 0; c4 < D / 4; ++c4) {
-        const float4 kv[2] = {__ldg(kp[0] + c4), __ldg(kp[1] + c4)};
-        step(c4, kv);
-      }
-      float* lo = m == 0 ? la : lm;
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int j = tid + i * KL;
-        if (j >= N) continue;
-#pragma unroll
-        for (int p = 0; p < R / 2; ++p) {
-          float a0, a1;
-          upk2f(acc[i][p], a0, a1);
-          lo[(2 * p) * N + j] = fmaf(g.sm_scale, a0, lc[i]);
-          lo[(2 * p + 1) * N + j] = fmaf(g.sm_scale, a1, lc[i]);
-        }
-      }
-    }
-  }
+  tc::fence_before_sync();
   __syncthreads();
-  rank_rows(g, w, la, lm, hist, bh, i0, rows, warp, lane, blockDim.x / 32);
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_holder;
+  const uint32_t idesc = idesc_tf32(kTcRows, kTcKeys);
+  const int rvalid = N - i0;                             // query rows of this CTA that exist
+  uint32_t stage_uses[2] = {0u, 0u};
+  int next_out = 0;                                      // next tile (0 .. 2 nt) to read out
+
+  // read the accumulator of tile v (map v / nt, key tile t0 + v % nt) out to the scratch:
+  // warp w reads TMEM lane quarter w % 4, columns 64 (w / 4) .. + 63 of the tile's buffer
+  auto read_out = [&](int v) {
+    const int buf = v & 1, m = v / nt, t = t0 + v % nt;
+    draft_wait(&bars[2 + buf], (uint32_t)(v >> 1) & 1u, w.err, g.wait_ns);
+    tc::fence_after_sync();
+    const int q = warp & 3, half = warp >> 2;
+    const int row = i0 + 32 * q + lane;
+    float* out = dlog + (((size_t)bh * N + row) * 2 + m) * NP;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      uint32_t r[32];
+      const int col = 64 * half + 32 * cc;
+      tc::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * kTcKeys + col), r);
+      tc::tmem_wait_ld();
+      const int j0 = t * kTcKeys + col;
+      if (row < N) {
+        if (j0 + 32 <= N) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float4 o;
+            o.x = fmaf(g.sm_scale, __uint_as_float(r[e]), lcs[j0 + e]);
+            o.y = fmaf(g.sm_scale, __uint_as_float(r[e + 1]), lcs[j0 + e + 1]);
+            o.z = fmaf(g.sm_scale, __uint_as_float(r[e + 2]), lcs[j0 + e + 2]);
+            o.w = fmaf(g.sm_scale, __uint_as_float(r[e + 3]), lcs[j0 + e + 3]);
+            *reinterpret_cast<float4*>(out + j0 + e) = o;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (j0 + e < N) out[j0 + e] = fmaf(g.sm_scale, __uint_as_float(r[e]), lcs[j0 + e]);
+        }
+      }
+    }
+    tc::fence_before_sync();
+  };
+
+  for (int m = 0; m < 2; ++m) {
+    const float* qsrc = (m == 0 ? w.qavg : w.qmax) + ((size_t)bh * N + i0) * D;
+    const float* ksrc = (m == 0 ? w.kavg : w.kmax) + (size_t)bh * N * D;
+    if (m == 1) {
+      // the queries of map 0 are read by every MMA issued so far: drain them first
+      while (next_out < nt) read_out(next_out++);
+      __syncthreads();
+    }
+    // queries of this map: 16 row groups x D/16 float4 groups, blocks of 8 rows x 4 float4
+    for (int b = warp; b < (kTcRows / 8) * (D / 16); b += kTcThreads / 32)
+      stage_split(qsrc, D, (b % (kTcRows / 8)) * 8, rvalid, (b / (kTcRows / 8)) * 4, a_hi, a_lo,
+                  D * 4, lane);
+    fence_async_smem();
+    __syncthreads();
+    for (int tt = 0; tt < nt; ++tt) {
+      const int u = m * nt + tt, buf = u & 1, t = t0 + tt;
+      const int kvalid = N - t * kTcKeys;
+      for (int kc = 0; kc < NKC; ++kc) {
+        const int si = (u * NKC + kc) & 1;
+        if (stage_uses[si] > 0) draft_wait(&bars[si], (stage_uses[si] - 1) & 1u, w.err, g.wait_ns);
+        uint8_t* bh_hi = b_st + si * 2 * B_PART;
+        uint8_t* bh_lo = bh_hi + B_PART;
+        // keys t*128 .. +127, channels 32 kc .. +31: 16 row groups x 2 float4 groups
+        for (int b = warp; b < (kTcKeys / 8) * (kTcKC / 16); b += kTcThreads / 32)
+          stage_split(ksrc + (size_t)t * kTcKeys * D + kc * kTcKC, D, (b % (kTcKeys / 8)) * 8, kvalid,
+                      (b / (kTcKeys / 8)) * 4, bh_hi, bh_lo, kTcKC * 4, lane);
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+          tc::fence_after_sync();
+          const uint32_t d_tmem = tmem + (uint32_t)(buf * kTcKeys);
+#pragma unroll
+          for (int ks = 0; ks < kTcKC / 8; ++ks) {
+            const uint32_t ka = (uint32_t)(kc * (kTcKC / 8) + ks) * 256u;   // 8 channels = 32 bytes
+            const uint64_t ah = tc::sdesc(a_hi + ka, 128, D * 4 * 8), al = tc::sdesc(a_lo + ka, 128, D * 4 * 8);
+            const uint64_t bhd = tc::sdesc(bh_hi + ks * 256, 128, kTcKC * 4 * 8),
+                           bld = tc::sdesc(bh_lo + ks * 256, 128, kTcKC * 4 * 8);
+            mma_tf32(d_tmem, ah, bhd, idesc, (kc | ks) != 0 ? 1u : 0u);
+            mma_tf32(d_tmem, ah, bld, idesc, 1u);
+            mma_tf32(d_tmem, al, bhd, idesc, 1u);
+          }
+          tc::mma_commit(&bars[si]);
+          if (kc == NKC - 1) tc::mma_commit(&bars[2 + buf]);
+        }
+        ++stage_uses[si];
+      }
+      // read out the previous tile while this one's MMAs run (its buffer is reused two
+      // tiles later, after the staging barriers of the next tile)
+      if (next_out < u) read_out(next_out++);
+    }
+  }
+  while (next_out < 2 * nt) read_out(next_out++);
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 2 * kTcKeys);
+  }
 }
 
-size_t tiled_smem_bytes(const Geo& g) {
-  return (size_t)(2 * g.d * kTileRows + 2 * kTileRows * g.N) * 4 + (size_t)kDraftWarps * 256 * 4;
+size_t logits_tc_smem_bytes(int d) {
+  return (size_t)2 * kTcRows * d * 4 + (size_t)4 * kTcKeys * kTcKC * 4 + 1024 * 4 + 4 * 8;
+}
+
+// Ranking of the draft scores from the logits scratch: 8 query blocks per CTA, one warp each,
+// the same per-row ranking as the other kernels (their two logit rows copied into shared
+// memory first).
+constexpr int kRankRows = 8;
+__global__ void __launch_bounds__(kRankRows * 32) k_draft_rank(Geo g, Ws w, const float* dlog, int NP) {
+  extern __shared__ __align__(16) float rsm[];
+  const int N = g.N;
+  float* la = rsm;                                      // [rows][N]
+  float* lm = la + kRankRows * N;                       // [rows][N]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(lm + kRankRows * N);   // [warps][256]
+  const int bh = blockIdx.y, i0 = blockIdx.x * kRankRows;
+  const int rows = min(kRankRows, N - i0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < rows) {
+    const float* src = dlog + ((size_t)bh * N + i0 + warp) * 2 * NP;
+    for (int j = lane; j < N; j += 32) {
+      la[warp * N + j] = src[j];
+      lm[warp * N + j] = src[NP + j];
+    }
+  }
+  __syncwarp();
+  rank_rows(g, w, la, lm, hist, bh, i0, rows, warp, lane, kRankRows);
+}
+
+size_t rank_smem_bytes(const Geo& g) {
+  return (size_t)2 * kRankRows * g.N * 4 + (size_t)kRankRows * 256 * 4;
 }
 
 size_t draft_smem_bytes(const Geo& g, int R) {
@@ -371,26 +486,29 @@ int draft_rows_per_cta(const Geo& g) {
   return R;
 }
 
-cudaError_t launch_draft_select(const Geo& g, const Ws& w, cudaStream_t st) {
-  // up to 1024 key blocks (and shared memory to spare): the register-tiled kernel
-  if (g.N <= 2 * kDraftThreads && tiled_smem_bytes(g) <= 232448) {
-    const int KL = kDraftThreads;                  // 16 warps: one per query row when ranking
-    const size_t smem = tiled_smem_bytes(g);
-    dim3 grid((g.N + kTileRows - 1) / kTileRows, g.B * g.H);
+cudaError_t launch_draft_select(const Geo& g, const Ws& w, float* dlog, int np, cudaStream_t st) {
+  // up to 1024 key blocks: the logits on the tensor cores into the scratch, then the ranking
+  if (g.N <= 1024) {
+    const int NT = (g.N + kTcKeys - 1) / kTcKeys;
+    const int per = NT < 2 ? NT : 2;                     // key tiles per CTA
+    const dim3 g1((g.N + kTcRows - 1) / kTcRows, g.B * g.H, (NT + per - 1) / per);
+    const size_t s1 = logits_tc_smem_bytes(g.d);
     cudaError_t e;
     if (g.d == 128) {
-      e = cudaFuncSetAttribute(k_draft_tiled<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      e = cudaFuncSetAttribute(k_draft_logits_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
       if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(k_draft_tiled<128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-      if (e != cudaSuccess) return e;
-      k_draft_tiled<128><<<grid, KL, smem, st>>>(g, w);
+      k_draft_logits_tc<128><<<g1, kTcThreads, s1, st>>>(g, w, dlog, np, per);
     } else {
-      e = cudaFuncSetAttribute(k_draft_tiled<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      e = cudaFuncSetAttribute(k_draft_logits_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
       if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(k_draft_tiled<64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-      if (e != cudaSuccess) return e;
-      k_draft_tiled<64><<<grid, KL, smem, st>>>(g, w);
+      k_draft_logits_tc<64><<<g1, kTcThreads, s1, st>>>(g, w, dlog, np, per);
     }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t s2 = rank_smem_bytes(g);
+    e = cudaFuncSetAttribute(k_draft_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
+    if (e != cudaSuccess) return e;
+    k_draft_rank<<<dim3((g.N + kRankRows - 1) / kRankRows, g.B * g.H), kRankRows * 32, s2, st>>>(g, w, dlog, np);
     return cudaGetLastError();
   }
   const int R = draft_rows_per_cta(g);
