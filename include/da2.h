@@ -148,6 +148,11 @@ typedef enum da2_status {
      dlog     fp32 [BH][N][2][np] the two draft logit rows (average map, max map) of every
               query block, written and read by da2_draft_select (scratch; size 0 when
               N > 1024).
+     qt, kt   the pooled Q and K of qavg/qmax and kavg/kmax again, each value split into a
+              tf32 high part and its fp32 remainder and laid out as the draft MMAs' operands:
+              per (b, h), 128-block tile, map (average, max) and 16-channel chunk, an 8 KB hi
+              part then an 8 KB lo part of 128 rows x 16 channels in the K-major core-matrix
+              layout (written by da2_prepare, read by da2_draft_select; size 0 when N > 1024).
      err      u32 device error word (0 = no error): bit 1 a bounded wait ran out, bit 2 an
               index or count of the selection was out of range, bit 4 a guard region of
               DA2_FLAG_DEBUG_CANARY was overwritten.
@@ -167,6 +172,7 @@ typedef struct da2_views {
   int n4max;            /* FP4 list length (n4 unless the adaptive budget is on) */
   size_t dlog;          /* draft logits scratch (N <= 1024), see below */
   int np;               /* its row length: N rounded up to a multiple of 4 */
+  size_t qt, kt;        /* pooled Q / K split for the draft MMAs (N <= 1024), see below */
 } da2_views;
 
 /* Workspace bytes needed for `cfg` (host only, no CUDA call). */

@@ -54,7 +54,8 @@ _VIEW_SIZES = ("tile8_qk", "tile4_qk", "tile8_v", "tile4_v", "sf_qk", "sf_v",
 class Views(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in _VIEW_INTS] + [(n, ctypes.c_size_t) for n in _VIEW_SIZES] + \
                [("nm", ctypes.c_int), ("listm", ctypes.c_size_t), ("n4max", ctypes.c_int),
-                ("dlog", ctypes.c_size_t), ("np", ctypes.c_int)]
+                ("dlog", ctypes.c_size_t), ("np", ctypes.c_int), ("qt", ctypes.c_size_t),
+                ("kt", ctypes.c_size_t)]
 
 
 class DA2Error(RuntimeError):
@@ -150,7 +151,7 @@ def workspace_size(cfg: Config) -> int:
 def workspace_views(cfg: Config) -> dict:
     v = Views()
     _check("da2_workspace_views", lib().da2_workspace_views(ctypes.byref(cfg), ctypes.byref(v)))
-    return {n: getattr(v, n) for n in _VIEW_INTS + _VIEW_SIZES + ("nm", "listm", "n4max", "dlog", "np")}
+    return {n: getattr(v, n) for n in _VIEW_INTS + _VIEW_SIZES + ("nm", "listm", "n4max", "dlog", "np", "qt", "kt")}
 
 
 def prepare(cfg, q, k, v, ws, stream=None):

@@ -6,11 +6,13 @@
 
 #include "checks.cuh"
 #include "common.cuh"
+#include "split_tiles.cuh"
 
 namespace da2 {
 cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
-                           const void* v, cudaStream_t st);
-cudaError_t launch_draft_select(const Geo& g, const Ws& w, float* dlog, int np, cudaStream_t st);
+                           const void* v, uint8_t* qt, uint8_t* kt, cudaStream_t st);
+cudaError_t launch_draft_select(const Geo& g, const Ws& w, const uint8_t* qt, const uint8_t* kt,
+                                float* dlog, int np, cudaStream_t st);
 cudaError_t launch_attention_tc(const Geo& g, const Ws& w, void* out, cudaStream_t st);
 da2_status noalloc_scratch(void** ptr, size_t* bytes);   // da2_noalloc.cu
 }  // namespace da2
@@ -113,6 +115,8 @@ void fill_views(const da2_config* c, da2_views* v, GuardList* gl = nullptr) {
   v->scores = take((c->flags & DA2_FLAG_EXPORT_SCORES) ? BH * N * N * 4 : 0);
   v->np = (int)((N + 3) / 4 * 4);
   v->dlog = take(N <= 1024 ? BH * N * 2 * (size_t)v->np * 4 : 0);
+  v->qt = take(N <= 1024 ? split_region_bytes((int)BH, (int)N, (int)d) : 0);
+  v->kt = take(N <= 1024 ? split_region_bytes((int)BH, (int)N, (int)d) : 0);
   v->err = take(4);
   v->total = off;
 }
@@ -240,7 +244,10 @@ da2_status da2_prepare(const da2_config* cfg, const void* q, const void* k, cons
   if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return DA2_ERR_ALIGNMENT;
   cudaError_t e = cudaSuccess;
   if (cfg->flags & DA2_FLAG_DEBUG_CANARY) e = launch_guards(static_cast<uint8_t*>(ws), gl, false, w.err, stream);
-  if (e == cudaSuccess) e = launch_prepare(g, w, q, k, v, stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* qt = g.N <= 1024 ? base + vw.qt : nullptr;
+  uint8_t* kt = g.N <= 1024 ? base + vw.kt : nullptr;
+  if (e == cudaSuccess) e = launch_prepare(g, w, q, k, v, qt, kt, stream);
   return finish_stage(cfg, w, ws, gl, e, stream);
 }
 
@@ -249,8 +256,9 @@ da2_status da2_draft_select(const da2_config* cfg, void* ws, size_t ws_bytes, cu
   da2_views vw; Geo g; Ws w; GuardList gl;
   const da2_status s = setup(cfg, ws, ws_bytes, &vw, &g, &w, &gl);
   if (s != DA2_OK) return s;
-  float* dlog = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + vw.dlog);
-  cudaError_t e = launch_draft_select(g, w, dlog, vw.np, stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* dlog = reinterpret_cast<float*>(base + vw.dlog);
+  cudaError_t e = launch_draft_select(g, w, base + vw.qt, base + vw.kt, dlog, vw.np, stream);
 #ifdef DA2_DEBUG
   if (e == cudaSuccess) e = launch_check_lists(g, w, stream);
 #endif

@@ -15,6 +15,7 @@
 // ascending index lists of the kept classes (FP8, mixed, FP4). Above 1024 key blocks one
 // kernel (k_draft_select) forms the logits with fp32 FMAs and ranks in the same way.
 #include "common.cuh"
+#include "split_tiles.cuh"
 #include "tc.cuh"
 
 namespace da2 {
@@ -236,19 +237,19 @@ __global__ void __launch_bounds__(kDraftThreads) k_draft_select(Geo g, Ws w, int
 }
 
 // ---- draft logits on the tensor cores (N <= 1024) ----
-// The two draft maps are dense contractions per head, L_map = Q_map K_map^T ([N, d] x [d, N]).
-// They run as tcgen05 MMAs of kind::tf32. A tf32 operand keeps 10 of fp32's 23 mantissa
-// bits, so each operand x is split into hi = x with its low 13 mantissa bits cleared (exact
-// in tf32) and lo = x - hi (exact in fp32, 13 significant bits of which tf32 keeps 10), and
-// each K step accumulates hi_a hi_b + hi_a lo_b + lo_a hi_b in fp32: every product of tf32
-// significands is exact, the dropped lo_a lo_b and lo's truncation are below 2^-20 of |a b|.
+// The two draft maps are dense contractions per head, L_map = Q_map K_map^T ([N, d] x [d, N]),
+// run as tcgen05 MMAs of kind::tf32 on operands that the preparation kernel has already split
+// into tf32 high parts and their remainders and laid out in the MMA's core-matrix chunks
+// (split_tiles.cuh); each K step of 8 channels accumulates hi_a hi_b + hi_a lo_b + lo_a hi_b
+// in fp32 (every product of tf32 significands is exact; the dropped lo_a lo_b and the
+// remainders' truncation to tf32 stay below 2^-20 of |a b|).
 // One CTA takes 128 query blocks (TMEM lanes) of one (b, h) and a range of 128-key tiles,
-// one map after the other: the queries of the map (both parts, K-major core-matrix layout,
-// all d channels) stay in shared memory, the keys stream in 32-channel stages (double
-// buffered), the accumulator of a tile sits in one of two 128-column TMEM buffers while the
-// other one is read out. The logits (sm_scale * acc + ln c_j) go to a global scratch of
-// [B*H][N][2][NP] fp32 rows that the ranking kernel reads.
-constexpr int kTcRows = 128, kTcKeys = 128, kTcKC = 32, kTcThreads = 256;
+// one map after the other. Warp 0 (one thread) bulk-copies the map's query chunks once and
+// the key chunks through a four-stage ring; warp 1 (one thread) issues the MMAs into one of
+// two 128-column TMEM accumulators; warps 2-5 (TMEM lane quarters 2, 3, 0, 1) read a finished
+// accumulator out as logits sm_scale * acc + ln c_j into the [B*H][N][2][np] fp32 scratch
+// that the ranking kernel reads.
+constexpr int kTcRows = 128, kTcKeys = 128, kTcStages = 4, kTcThreads = 192;
 
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
   // D fp32, A and B tf32, both K-major, N / 8, M / 16
@@ -261,71 +262,67 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ unsigned long long draft_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait on an mbarrier phase; a wait that runs out sets the error word and returns.
-__device__ __forceinline__ void draft_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+// Bounded wait on an mbarrier phase; a wait that runs out sets the error word and returns
+// false (the caller stops issuing work).
+__device__ __forceinline__ bool draft_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
                                            unsigned long long limit_ns) {
-  if (tc::mbar_try_wait(bar, parity)) return;
+  if (tc::mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = draft_ns();
   while (!tc::mbar_try_wait(bar, parity)) {
     if (draft_ns() - t0 > limit_ns) {
       set_error(err, kErrWaitTimeout);
-      return;
+      return false;
     }
   }
-}
-// tf32 high part (low 13 mantissa bits cleared) and the exact remainder.
-__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
-  hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
-  lo = x - hi;
-}
-// 8 rows x 4 float4 of a row-major fp32 [rows][D] source into the hi and lo tiles (K-major
-// core matrices: rows of `rowbytes` bytes); lane l takes row r0 + (l & 7), float4 c0 + (l >> 3),
-// so a warp reads 8 x 64 contiguous bytes and writes 512 contiguous bytes of each tile.
-__device__ __forceinline__ void stage_split(const float* src, int ld, int r0, int rvalid, int c0,
-                                            uint8_t* hi, uint8_t* lo, uint32_t rowbytes, int lane) {
-  const int r = r0 + (lane & 7), c4 = c0 + (lane >> 3);
-  float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  if (r < rvalid) x = __ldg(reinterpret_cast<const float4*>(src + (size_t)r * ld) + c4);
-  float4 h, l;
-  split_tf32(x.x, h.x, l.x);
-  split_tf32(x.y, h.y, l.y);
-  split_tf32(x.z, h.z, l.z);
-  split_tf32(x.w, h.w, l.w);
-  const uint32_t off = kmajor_off((uint32_t)r, (uint32_t)c4 * 16u, rowbytes);
-  *reinterpret_cast<float4*>(hi + off) = h;
-  *reinterpret_cast<float4*>(lo + off) = l;
+  return true;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1) k_draft_logits_tc(Geo g, Ws w, float* dlog, int NP, int tiles_per_cta) {
-  constexpr uint32_t A_PART = kTcRows * D * 4;          // one part of the queries, all channels
-  constexpr uint32_t B_PART = kTcKeys * kTcKC * 4;      // one part of a key stage
-  constexpr int NKC = D / kTcKC;                        // key stages per tile
+__global__ void __launch_bounds__(kTcThreads, 1) k_draft_logits_tc(Geo g, Ws w, const uint8_t* __restrict__ qt,
+                                                                  const uint8_t* __restrict__ kt,
+                                                                  float* dlog, int NP, int tiles_per_cta) {
+  constexpr int NKC = D / kSplitKC;                       // 16-channel chunks
+  constexpr uint32_t CHUNK = 2 * kSplitPart;              // hi + lo of one chunk, 16 KB
+  constexpr uint32_t A_BYTES = NKC * CHUNK;               // all chunks of the queries
   extern __shared__ __align__(1024) uint8_t dsm_tc[];
-  uint8_t* a_hi = dsm_tc;
-  uint8_t* a_lo = dsm_tc + A_PART;
-  uint8_t* b_st = dsm_tc + 2 * A_PART;                  // [stage][part][B_PART]
-  float* lcs = reinterpret_cast<float*>(b_st + 4 * B_PART);          // ln c_j, [1024]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(lcs + 1024);           // stage_free[2], acc_full[2]
+  uint8_t* a_sm = dsm_tc;                                 // [kc][part][8 KB]
+  uint8_t* b_sm = dsm_tc + A_BYTES;                       // [stage][part][8 KB]
+  float* lcs = reinterpret_cast<float*>(b_sm + kTcStages * CHUNK);   // ln c_j, [1024]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(lcs + 1024);
+  uint64_t* a_full = bars;                                // queries of the map in place
+  uint64_t* a_empty = bars + 1;                           // MMAs done with them
+  uint64_t* b_full = bars + 2;                            // [kTcStages]
+  uint64_t* b_empty = b_full + kTcStages;                 // [kTcStages]
+  uint64_t* acc_full = b_empty + kTcStages;               // [2]
+  uint64_t* acc_empty = acc_full + 2;                     // [2]
   __shared__ uint32_t tmem_holder;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int N = g.N, bh = blockIdx.y, i0 = blockIdx.x * kTcRows;
+  const int N = g.N, bh = blockIdx.y, rtile = blockIdx.x, i0 = rtile * kTcRows;
+  const int RT = (N + kSplitRows - 1) / kSplitRows;
   const int NT = (N + kTcKeys - 1) / kTcKeys;
   const int t0 = blockIdx.z * tiles_per_cta, t1 = min(NT, t0 + tiles_per_cta);
   if (t0 >= t1) return;
-  const int nt = t1 - t0;
+  const int nt = t1 - t0, U = 2 * nt;                     // accumulator tiles of this CTA
   if (warp == 0) {
     tc::tmem_alloc(&tmem_holder, 2 * kTcKeys);
     tc::tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
+    tc::mbar_init(a_full, 1);
+    tc::mbar_init(a_empty, 1);
+    for (int i = 0; i < kTcStages; ++i) {
+      tc::mbar_init(&b_full[i], 1);
+      tc::mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&acc_full[i], 1);
+      tc::mbar_init(&acc_empty[i], 4);                    // one arrival per read-out warp
+    }
     tc::fence_mbar_init();
   }
   const bool mass = !(g.flags & DA2_FLAG_NO_MASS_CORRECTION);
@@ -343,100 +340,106 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_draft_logits_tc(Geo g, Ws w, 
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_holder;
-  const uint32_t idesc = idesc_tf32(kTcRows, kTcKeys);
-  const int rvalid = N - i0;                             // query rows of this CTA that exist
-  uint32_t stage_uses[2] = {0u, 0u};
-  int next_out = 0;                                      // next tile (0 .. 2 nt) to read out
 
-  // read the accumulator of tile v (map v / nt, key tile t0 + v % nt) out to the scratch:
-  // warp w reads TMEM lane quarter w % 4, columns 64 (w / 4) .. + 63 of the tile's buffer
-  auto read_out = [&](int v) {
-    const int buf = v & 1, m = v / nt, t = t0 + v % nt;
-    draft_wait(&bars[2 + buf], (uint32_t)(v >> 1) & 1u, w.err, g.wait_ns);
-    tc::fence_after_sync();
-    const int q = warp & 3, half = warp >> 2;
-    const int row = i0 + 32 * q + lane;
-    float* out = dlog + (((size_t)bh * N + row) * 2 + m) * NP;
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      uint32_t r[32];
-      const int col = 64 * half + 32 * cc;
-      tc::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * kTcKeys + col), r);
-      tc::tmem_wait_ld();
-      const int j0 = t * kTcKeys + col;
-      if (row < N) {
-        if (j0 + 32 <= N) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float4 o;
-            o.x = fmaf(g.sm_scale, __uint_as_float(r[e]), lcs[j0 + e]);
-            o.y = fmaf(g.sm_scale, __uint_as_float(r[e + 1]), lcs[j0 + e + 1]);
-            o.z = fmaf(g.sm_scale, __uint_as_float(r[e + 2]), lcs[j0 + e + 2]);
-            o.w = fmaf(g.sm_scale, __uint_as_float(r[e + 3]), lcs[j0 + e + 3]);
-            *reinterpret_cast<float4*>(out + j0 + e) = o;
+  if (warp == 0) {
+    // ---- copies: per map the query chunks, then the key chunks of every tile ----
+    if (lane == 0) {
+      int idx = 0;
+      for (int m = 0; m < 2; ++m) {
+        if (m > 0 && !draft_wait(a_empty, 0, w.err, g.wait_ns)) break;
+        tc::mbar_arrive_expect_tx(a_full, A_BYTES);
+        for (int kc = 0; kc < NKC; ++kc)
+          tc::bulk_g2s(a_sm + kc * CHUNK, qt + split_chunk_off(bh, RT, rtile, m, kc, NKC), CHUNK, a_full);
+        bool ok = true;
+        for (int tt = 0; tt < nt && ok; ++tt)
+          for (int kc = 0; kc < NKC; ++kc, ++idx) {
+            const int s = idx % kTcStages;
+            if (idx >= kTcStages && !draft_wait(&b_empty[s], (uint32_t)(idx / kTcStages - 1) & 1u, w.err, g.wait_ns)) {
+              ok = false;
+              break;
+            }
+            tc::mbar_arrive_expect_tx(&b_full[s], CHUNK);
+            tc::bulk_g2s(b_sm + s * CHUNK, kt + split_chunk_off(bh, RT, t0 + tt, m, kc, NKC), CHUNK, &b_full[s]);
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (j0 + e < N) out[j0 + e] = fmaf(g.sm_scale, __uint_as_float(r[e]), lcs[j0 + e]);
-        }
+        if (!ok) break;
       }
     }
-    tc::fence_before_sync();
-  };
-
-  for (int m = 0; m < 2; ++m) {
-    const float* qsrc = (m == 0 ? w.qavg : w.qmax) + ((size_t)bh * N + i0) * D;
-    const float* ksrc = (m == 0 ? w.kavg : w.kmax) + (size_t)bh * N * D;
-    if (m == 1) {
-      // the queries of map 0 are read by every MMA issued so far: drain them first
-      while (next_out < nt) read_out(next_out++);
-      __syncthreads();
-    }
-    // queries of this map: 16 row groups x D/16 float4 groups, blocks of 8 rows x 4 float4
-    for (int b = warp; b < (kTcRows / 8) * (D / 16); b += kTcThreads / 32)
-      stage_split(qsrc, D, (b % (kTcRows / 8)) * 8, rvalid, (b / (kTcRows / 8)) * 4, a_hi, a_lo,
-                  D * 4, lane);
-    fence_async_smem();
-    __syncthreads();
-    for (int tt = 0; tt < nt; ++tt) {
-      const int u = m * nt + tt, buf = u & 1, t = t0 + tt;
-      const int kvalid = N - t * kTcKeys;
-      for (int kc = 0; kc < NKC; ++kc) {
-        const int si = (u * NKC + kc) & 1;
-        if (stage_uses[si] > 0) draft_wait(&bars[si], (stage_uses[si] - 1) & 1u, w.err, g.wait_ns);
-        uint8_t* bh_hi = b_st + si * 2 * B_PART;
-        uint8_t* bh_lo = bh_hi + B_PART;
-        // keys t*128 .. +127, channels 32 kc .. +31: 16 row groups x 2 float4 groups
-        for (int b = warp; b < (kTcKeys / 8) * (kTcKC / 16); b += kTcThreads / 32)
-          stage_split(ksrc + (size_t)t * kTcKeys * D + kc * kTcKC, D, (b % (kTcKeys / 8)) * 8, kvalid,
-                      (b / (kTcKeys / 8)) * 4, bh_hi, bh_lo, kTcKC * 4, lane);
-        fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {
+  } else if (warp == 1) {
+    // ---- MMAs: 3 per K step of 8 channels, 6 per 16-channel chunk ----
+    if (lane == 0) {
+      const uint32_t idesc = idesc_tf32(kTcRows, kTcKeys);
+      int idx = 0;
+      bool ok = true;
+      for (int m = 0; m < 2 && ok; ++m) {
+        ok = draft_wait(a_full, (uint32_t)m & 1u, w.err, g.wait_ns);
+        tc::fence_after_sync();
+        for (int tt = 0; tt < nt && ok; ++tt) {
+          const int u = m * nt + tt, buf = u & 1;
+          if (u >= 2 && !(ok = draft_wait(&acc_empty[buf], (uint32_t)((u >> 1) - 1) & 1u, w.err, g.wait_ns))) break;
           tc::fence_after_sync();
           const uint32_t d_tmem = tmem + (uint32_t)(buf * kTcKeys);
+          for (int kc = 0; kc < NKC; ++kc, ++idx) {
+            const int s = idx % kTcStages;
+            if (!(ok = draft_wait(&b_full[s], (uint32_t)(idx / kTcStages) & 1u, w.err, g.wait_ns))) break;
+            tc::fence_after_sync();
+            const uint8_t* ah = a_sm + kc * CHUNK;
+            const uint8_t* bhp = b_sm + s * CHUNK;
 #pragma unroll
-          for (int ks = 0; ks < kTcKC / 8; ++ks) {
-            const uint32_t ka = (uint32_t)(kc * (kTcKC / 8) + ks) * 256u;   // 8 channels = 32 bytes
-            const uint64_t ah = tc::sdesc(a_hi + ka, 128, D * 4 * 8), al = tc::sdesc(a_lo + ka, 128, D * 4 * 8);
-            const uint64_t bhd = tc::sdesc(bh_hi + ks * 256, 128, kTcKC * 4 * 8),
-                           bld = tc::sdesc(bh_lo + ks * 256, 128, kTcKC * 4 * 8);
-            mma_tf32(d_tmem, ah, bhd, idesc, (kc | ks) != 0 ? 1u : 0u);
-            mma_tf32(d_tmem, ah, bld, idesc, 1u);
-            mma_tf32(d_tmem, al, bhd, idesc, 1u);
+            for (int ks = 0; ks < kSplitKC / 8; ++ks) {
+              const uint64_t adh = tc::sdesc(ah + ks * 256, 128, kSplitKC * 4 * 8);
+              const uint64_t adl = tc::sdesc(ah + kSplitPart + ks * 256, 128, kSplitKC * 4 * 8);
+              const uint64_t bdh = tc::sdesc(bhp + ks * 256, 128, kSplitKC * 4 * 8);
+              const uint64_t bdl = tc::sdesc(bhp + kSplitPart + ks * 256, 128, kSplitKC * 4 * 8);
+              mma_tf32(d_tmem, adh, bdh, idesc, (kc | ks) != 0 ? 1u : 0u);
+              mma_tf32(d_tmem, adh, bdl, idesc, 1u);
+              mma_tf32(d_tmem, adl, bdh, idesc, 1u);
+            }
+            tc::mma_commit(&b_empty[s]);
           }
-          tc::mma_commit(&bars[si]);
-          if (kc == NKC - 1) tc::mma_commit(&bars[2 + buf]);
+          if (ok) tc::mma_commit(&acc_full[buf]);
         }
-        ++stage_uses[si];
+        if (ok) tc::mma_commit(a_empty);                  // this map's MMAs are all issued
       }
-      // read out the previous tile while this one's MMAs run (its buffer is reused two
-      // tiles later, after the staging barriers of the next tile)
-      if (next_out < u) read_out(next_out++);
+    }
+  } else {
+    // ---- read-out: warp w owns TMEM lanes 32 (w % 4) .. + 31, i.e. query rows ----
+    const int q = warp & 3;
+    const int row = i0 + 32 * q + lane;
+    for (int u = 0; u < U; ++u) {
+      const int buf = u & 1, m = u / nt, t = t0 + u % nt;
+      if (!draft_wait(&acc_full[buf], (uint32_t)(u >> 1) & 1u, w.err, g.wait_ns)) break;
+      tc::fence_after_sync();
+      float* out = dlog + (((size_t)bh * N + row) * 2 + m) * NP;
+#pragma unroll
+      for (int cc = 0; cc < kTcKeys / 32; ++cc) {
+        uint32_t r[32];
+        tc::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * kTcKeys + 32 * cc), r);
+        tc::tmem_wait_ld();
+        const int j0 = t * kTcKeys + 32 * cc;
+        if (row < N) {
+          if (j0 + 32 <= N) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              float4 o;
+              o.x = fmaf(g.sm_scale, __uint_as_float(r[e]), lcs[j0 + e]);
+              o.y = fmaf(g.sm_scale, __uint_as_float(r[e + 1]), lcs[j0 + e + 1]);
+              o.z = fmaf(g.sm_scale, __uint_as_float(r[e + 2]), lcs[j0 + e + 2]);
+              o.w = fmaf(g.sm_scale, __uint_as_float(r[e + 3]), lcs[j0 + e + 3]);
+              *reinterpret_cast<float4*>(out + j0 + e) = o;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (j0 + e < N) out[j0 + e] = fmaf(g.sm_scale, __uint_as_float(r[e]), lcs[j0 + e]);
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&acc_empty[buf]);
     }
   }
-  while (next_out < 2 * nt) read_out(next_out++);
+  tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
     tc::fence_after_sync();
@@ -445,7 +448,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_draft_logits_tc(Geo g, Ws w, 
 }
 
 size_t logits_tc_smem_bytes(int d) {
-  return (size_t)2 * kTcRows * d * 4 + (size_t)4 * kTcKeys * kTcKC * 4 + 1024 * 4 + 4 * 8;
+  return (size_t)(d / kSplitKC) * 2 * kSplitPart + (size_t)kTcStages * 2 * kSplitPart + 1024 * 4 + 16 * 8;
 }
 
 // Ranking of the draft scores from the logits scratch: 8 query blocks per CTA, one warp each,
@@ -486,7 +489,8 @@ int draft_rows_per_cta(const Geo& g) {
   return R;
 }
 
-cudaError_t launch_draft_select(const Geo& g, const Ws& w, float* dlog, int np, cudaStream_t st) {
+cudaError_t launch_draft_select(const Geo& g, const Ws& w, const uint8_t* qt, const uint8_t* kt,
+                                float* dlog, int np, cudaStream_t st) {
   // up to 1024 key blocks: the logits on the tensor cores into the scratch, then the ranking
   if (g.N <= 1024) {
     const int NT = (g.N + kTcKeys - 1) / kTcKeys;
@@ -497,11 +501,11 @@ cudaError_t launch_draft_select(const Geo& g, const Ws& w, float* dlog, int np, 
     if (g.d == 128) {
       e = cudaFuncSetAttribute(k_draft_logits_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
       if (e != cudaSuccess) return e;
-      k_draft_logits_tc<128><<<g1, kTcThreads, s1, st>>>(g, w, dlog, np, per);
+      k_draft_logits_tc<128><<<g1, kTcThreads, s1, st>>>(g, w, qt, kt, dlog, np, per);
     } else {
       e = cudaFuncSetAttribute(k_draft_logits_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
       if (e != cudaSuccess) return e;
-      k_draft_logits_tc<64><<<g1, kTcThreads, s1, st>>>(g, w, dlog, np, per);
+      k_draft_logits_tc<64><<<g1, kTcThreads, s1, st>>>(g, w, qt, kt, dlog, np, per);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -12,6 +12,7 @@
 // vectors (Q, K), the E4M3 copy and the E2M1 copy with its E4M3 group scales in the tile
 // layouts the attention kernel loads directly (see include/da2.h).
 #include "common.cuh"
+#include "split_tiles.cuh"
 
 namespace da2 {
 
@@ -219,7 +220,7 @@ __device__ __forceinline__ void stage_window(const Geo& g, const __nv_bfloat16* 
 
 // Q (which 0) or K (which 1) block n of head bh from the staged window.
 template <int D>
-__device__ __forceinline__ void qk_block(const Geo& g, const Ws& w, int which, int bh, int n,
+__device__ __forceinline__ void qk_block(const Geo& g, const Ws& w, uint8_t* tiles, int which, int bh, int n,
                                          const PrepSmem<D>& sm) {
   constexpr int RS = D + 8;
   const __nv_bfloat16* X = sm.X;
@@ -251,7 +252,9 @@ __device__ __forceinline__ void qk_block(const Geo& g, const Ws& w, int which, i
       for (int wx = 0; wx < wv; ++wx) acc_bf16x2(*reinterpret_cast<const uint32_t*>(row + wx * RS), a0, a1);
     }
     const float cnt = (float)(hv * wv);
-    *reinterpret_cast<float2*>(avg_out + c2) = make_float2(__fdiv_rn(a0, cnt), __fdiv_rn(a1, cnt));
+    const float x0 = __fdiv_rn(a0, cnt), x1 = __fdiv_rn(a1, cnt);
+    *reinterpret_cast<float2*>(avg_out + c2) = make_float2(x0, x1);
+    if (tiles) write_split_pair(tiles, bh, g.N, D, n, 0, c2, x0, x1);
   } else {
     const int mw = warp - NSW, ch = lane % CPW, sg = mw * SPW + lane / CPW;
     uint32_t mx[4], mn[4];
@@ -302,8 +305,9 @@ __device__ __forceinline__ void qk_block(const Geo& g, const Ws& w, int which, i
     uint32_t m2 = pmax[tid];
 #pragma unroll
     for (int k = 1; k < NMW; ++k) m2 = bmax2(m2, pmax[k * CPW * 4 + tid]);
-    *reinterpret_cast<float2*>(max_out + 2 * tid) =
-        make_float2(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+    const float x0 = __uint_as_float(m2 << 16), x1 = __uint_as_float(m2 & 0xFFFF0000u);
+    *reinterpret_cast<float2*>(max_out + 2 * tid) = make_float2(x0, x1);
+    if (tiles) write_split_pair(tiles, bh, g.N, D, n, 1, 2 * tid, x0, x1);
   }
   float am = wam[0];
 #pragma unroll
@@ -425,7 +429,7 @@ template <int D, bool BTHD>
 __global__ void __launch_bounds__(256) k_prepare_qk(Geo g, Ws w, const __nv_bfloat16* __restrict__ q,
                                                     const __nv_bfloat16* __restrict__ k,
                                                     const __nv_bfloat16* __restrict__ v,
-                                                    int chunk, int nc) {
+                                                    uint8_t* qt, uint8_t* kt, int chunk, int nc) {
   extern __shared__ __align__(16) uint8_t smem[];
   const PrepSmem<D> sm = prep_smem<D>(smem, g.bs);
   const int tid = threadIdx.x, N = g.N;
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(256) k_prepare_qk(Geo g, Ws w, const __nv_bflo
   if (tid < 128) sm.rcp_tab[tid] = tid > 0 ? __frcp_rn(e4m3_to_f32((uint8_t)tid)) : 0.0f;
   cp_async_wait_all();
   __syncthreads();
-  qk_block<D>(g, w, which, bh, n, sm);
+  qk_block<D>(g, w, which == 0 ? qt : kt, which, bh, n, sm);
 }
 
 // Second kernel: V block blockIdx.x of head blockIdx.y.
@@ -470,7 +474,7 @@ size_t prepare_smem_bytes(const Geo& g) {
 constexpr int kAmaxChunk = 1024;
 
 cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void* k,
-                           const void* v, cudaStream_t st) {
+                           const void* v, uint8_t* qt, uint8_t* kt, cudaStream_t st) {
   const int BH = g.B * g.H;
   cudaError_t e = cudaMemsetAsync(w.vamax, 0, sizeof(float) * BH * g.d, st);
   if (e != cudaSuccess) return e;
@@ -483,16 +487,16 @@ cudaError_t launch_prepare(const Geo& g, const Ws& w, const void* q, const void*
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
   const auto* vb = static_cast<const __nv_bfloat16*>(v);
   if (g.d == 128 && !g.bthd) {
-    k_prepare_qk<128, false><<<g1, 256, smem, st>>>(g, w, qb, kb, vb, kAmaxChunk, nc);
+    k_prepare_qk<128, false><<<g1, 256, smem, st>>>(g, w, qb, kb, vb, qt, kt, kAmaxChunk, nc);
     k_prepare_v<128, false><<<g2, 256, smem, st>>>(g, w, vb);
   } else if (g.d == 128) {
-    k_prepare_qk<128, true><<<g1, 256, smem, st>>>(g, w, qb, kb, vb, kAmaxChunk, nc);
+    k_prepare_qk<128, true><<<g1, 256, smem, st>>>(g, w, qb, kb, vb, qt, kt, kAmaxChunk, nc);
     k_prepare_v<128, true><<<g2, 256, smem, st>>>(g, w, vb);
   } else if (!g.bthd) {
-    k_prepare_qk<64, false><<<g1, 256, smem, st>>>(g, w, qb, kb, vb, kAmaxChunk, nc);
+    k_prepare_qk<64, false><<<g1, 256, smem, st>>>(g, w, qb, kb, vb, qt, kt, kAmaxChunk, nc);
     k_prepare_v<64, false><<<g2, 256, smem, st>>>(g, w, vb);
   } else {
-    k_prepare_qk<64, true><<<g1, 256, smem, st>>>(g, w, qb, kb, vb, kAmaxChunk, nc);
+    k_prepare_qk<64, true><<<g1, 256, smem, st>>>(g, w, qb, kb, vb, qt, kt, kAmaxChunk, nc);
     k_prepare_v<64, true><<<g2, 256, smem, st>>>(g, w, vb);
   }
   return cudaGetLastError();

@@ -160,7 +160,7 @@ def test_adaptive_budget_views_and_limits():
 
 
 REGIONS = ("q8", "k8", "v8", "q4", "k4", "v4", "sfq4", "sfk4", "sfv4", "sq", "sk", "sv", "vamax",
-           "qavg", "qmax", "kavg", "kmax", "tags", "list8", "list4", "listm", "dlog", "err")
+           "qavg", "qmax", "kavg", "kmax", "tags", "list8", "list4", "listm", "dlog", "qt", "kt", "err")
 
 
 @pytest.mark.parametrize("name", ["tiny", "wan720", "hunyuan720"])

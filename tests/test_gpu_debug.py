@@ -13,7 +13,7 @@ from sparse_mixed_precision_b200.synth import WORKLOADS, generate, scaled
 pytestmark = pytest.mark.gpu
 
 REGIONS = ("q8", "k8", "v8", "q4", "k4", "v4", "sfq4", "sfk4", "sfv4", "sq", "sk", "sv", "vamax",
-           "qavg", "qmax", "kavg", "kmax", "tags", "list8", "list4", "listm", "dlog", "err")
+           "qavg", "qmax", "kavg", "kmax", "tags", "list8", "list4", "listm", "dlog", "qt", "kt", "err")
 
 CASES = {
     "tiny": WORKLOADS["tiny"],
