@@ -175,6 +175,27 @@ def test_full_size_sampled_parity(name):
     assert torch.isfinite(out).all()
 
 
+def test_more_than_1024_key_blocks_uses_the_general_draft_kernel():
+    # 4x8-token windows on the Wan-480p frame: 21 x 8 x 7 = 1176 key blocks per head, above
+    # the tensor-core draft path's 1024; the fp32-FMA selection kernel runs instead
+    w = scaled(WORKLOADS["wan480"], name="wan480-w32", H=2, ph=4, pw=8)
+    g = O.geometry(scaled(w, B=1, H=1))
+    assert g.N > 1024
+    q, k, v = generate(w, device="cuda")
+    cfg, views, ws, out = run_cuda(w, q, k, v)
+    rd = WsReader(ws, views, w.d)
+    rng = np.random.default_rng(11)
+    edge = [i for i in range(g.N) if O.block_counts(g)[i] < g.bs]
+    for h in range(w.H):
+        qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+        P = check_prep(w, views, rd, h, qh, kh, vh)
+        l8, l4, _ = check_selection(views, rd, h, P, g)
+        blocks = sorted(set([0, g.N - 1] + list(rng.choice(g.N, 4, replace=False)) +
+                            (list(rng.choice(edge, 2, replace=False)) if edge else [])))
+        check_attention(w, views, P, l8[0], l4[0], out[0, h].float().cpu().numpy(), blocks, g)
+    assert torch.isfinite(out).all()
+
+
 def test_repeated_calls_are_deterministic():
     w = scaled(WORKLOADS["wan720"], F=3)
     q, k, v = generate(w, device="cuda")
