@@ -29,7 +29,15 @@ from sparse_mixed_precision_b200.synth import WORKLOADS, generate  # noqa: E402
 
 METRIC = "dense-equivalent TFLOP/s of one DraftAttention2 attention call (75.6k tokens)"
 UNIT = "TFLOP/s"
-KERNELS_PER_STEP = 4      # k_prepare_qk, k_prepare_v, draft selection, attention
+
+
+def kernels_per_step(w) -> int:
+    """Library kernels launched by one step: k_prepare_qk, k_prepare_v, the draft selection
+    (k_draft_logits_tc + k_draft_rank up to 1024 key blocks, else k_draft_select) and
+    k_attention_tc."""
+    import math as _m
+    N = w.F * _m.ceil(w.Hf / w.ph) * _m.ceil(w.Wf / w.pw)
+    return 5 if N <= 1024 else 4
 
 
 def dense_flops(w) -> float:
@@ -138,9 +146,22 @@ def tensor_roofline_ms(w, peaks: dict, sustained: bool = False) -> float:
     return (f8 / (2.0 * bf16 * 1e12) + f4 / (4.0 * bf16 * 1e12)) * 1e3
 
 
+def draft_tensor_entry(w, draft_ms: float, peaks: dict) -> dict:
+    """The draft stage against the tensor cores that run its logits (up to 1024 key blocks):
+    three kind::tf32 products per K step (operands split into tf32 high parts and
+    remainders) of the two (N x d) @ (d x N) maps per head, against the tf32 rate taken as
+    half the measured burst bf16 rate (NVIDIA's nominal dense 2.25 : 1.1 PFLOP/s). The stage
+    also ranks every row (instruction-bound), so the fraction is of the whole stage."""
+    tf32 = peaks.get("bf16_tflops", 1590.0) / 2.0
+    achieved = 3.0 * draft_flops(w) / (draft_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": tf32, "unit": "TFLOP/s",
+            "frac": achieved / tf32,
+            "note": "3 tf32 MMA products per K step; peak = measured burst bf16 / 2"}
+
+
 def draft_alu_entry(w, draft_ms: float, peaks: dict) -> dict:
-    """The draft stage against its own bound: fp32 FMA throughput (ALU-bound; it reads only
-    the 52 MB of pooled vectors), peak from the unit counts at the measured max SM clock."""
+    """The draft stage above 1024 key blocks against its bound: fp32 FMA throughput (the
+    logits on the FMA pipe), peak from the unit counts at the measured max SM clock."""
     peak = fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
     achieved = draft_flops(w) / (draft_ms * 1e-3) / 1e12
     return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -485,9 +506,10 @@ def main():
                              f" sustained bf16 rate, t_roof {t_roof_sus:.2f} ms)"},
         "prepare_hbm": hbm_entry(pb, prep_ms, peaks),
         "draft_hbm": hbm_entry(db, draft_ms, peaks),
-        "draft_alu": draft_alu_entry(w, draft_ms, peaks),
+        ("draft_tensor" if kernels_per_step(w) == 5 else "draft_alu"):
+            (draft_tensor_entry if kernels_per_step(w) == 5 else draft_alu_entry)(w, draft_ms, peaks),
         "step_roofline_frac": (t_roof + (pb + db) / (peaks["hbm_gbs"] * 1e9) * 1e3) / ms,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(w) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and args.heads == 0:

@@ -32,3 +32,13 @@ def test_draft_bytes_and_tensor_roofline():
         (f8 / 3311e12 + f4 / 6622e12) * 1e3)                      # 10.06 ms at the burst rate
     assert bench.tensor_roofline_ms(w, peaks) == pytest.approx(10.06, rel=2e-3)
     assert bench.tensor_roofline_ms(w, peaks, sustained=True) > bench.tensor_roofline_ms(w, peaks)
+
+
+def test_draft_tensor_bound_and_launch_count():
+    w = WORKLOADS["wan720"]
+    e = bench.draft_tensor_entry(w, 1.0, {"bf16_tflops": 1655.5})
+    assert e["bound"] == "tensor" and e["peak"] == pytest.approx(1655.5 / 2)
+    assert e["achieved"] == pytest.approx(3 * bench.draft_flops(w) / 1e-3 / 1e12)
+    assert bench.kernels_per_step(w) == 5                     # N = 630: two draft kernels
+    from sparse_mixed_precision_b200.synth import scaled
+    assert bench.kernels_per_step(scaled(WORKLOADS["wan480"], ph=4, pw=8)) == 4   # N = 1176
