@@ -494,7 +494,7 @@ cudaError_t launch_draft_select(const Geo& g, const Ws& w, const uint8_t* qt, co
   // up to 1024 key blocks: the logits on the tensor cores into the scratch, then the ranking
   if (g.N <= 1024) {
     const int NT = (g.N + kTcKeys - 1) / kTcKeys;
-    const int per = NT < 2 ? NT : 2;                     // key tiles per CTA
+    const int per = NT < 3 ? NT : 3;                     // key tiles per CTA (A/B: 3 beats 1, 2 and all)
     const dim3 g1((g.N + kTcRows - 1) / kTcRows, g.B * g.H, (NT + per - 1) / per);
     const size_t s1 = logits_tc_smem_bytes(g.d);
     cudaError_t e;
