@@ -131,3 +131,31 @@ def test_debug_build_matches_the_release_build(name):
         if r != "err":
             a0, a1 = sp[r]
             assert torch.equal(ws_r[a0:a1], ws_d[a0:a1]), r
+
+
+def test_debug_build_reports_a_set_error_word_at_the_call():
+    """A DA2_DEBUG stage call waits for its stream and returns DA2_ERR_TIMEOUT as soon as the
+    error word is set; the release build returns at once and leaves the word for
+    da2_get_error. The word is set by the host between two calls (the draft kernels only
+    ever set it, never read it)."""
+    w = WORKLOADS["tiny"]
+    cfg, ws, _ = run(w)
+    err = da2.workspace_views(cfg)["err"]
+
+    def draft_with_word_set():
+        ws[err:err + 4] = torch.tensor([1, 0, 0, 0], dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+        da2.draft_select(cfg, ws)
+        torch.cuda.synchronize()
+
+    draft_with_word_set()                                  # release build: no error raised
+    assert da2.get_error(cfg, ws) == 1                     # the word was left for get_error
+    prev = da2.use_library(da2.LIB_DEBUG_PATH)
+    try:
+        with pytest.raises(da2.DA2Error) as e:
+            draft_with_word_set()
+        assert e.value.status == 6
+        assert da2.get_error(cfg, ws) == 1                 # still set; get_error clears it
+        assert da2.get_error(cfg, ws) == 0
+    finally:
+        da2.use_library(prev)
