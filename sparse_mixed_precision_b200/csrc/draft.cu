@@ -73,16 +73,75 @@ __device__ void warp_radix_select(const uint32_t* keys, int n, int kth, uint32_t
 
 constexpr int kDraftThreads = 512, kDraftWarps = kDraftThreads / 32;
 
-// Per-row ranking of the draft scores (one warp per row): the two row softmaxes of the
-// average- and max-pooled logits (in la / lm, R rows of N), their mean as the score, and the
-// radix-select cuts of the shared ranking; writes tags and the ascending lists.
-__device__ void rank_rows(const Geo& g, const Ws& w, float* la, float* lm, uint32_t* hist, int bh, int i0,
-                          int rows, int warp, int lane, int nwarps) {
+// The shared ranking of one score row (one warp; keys = the N scores' bit patterns, which
+// order like the non-negative scores): the radix-select cuts, then tags and the ascending
+// lists of the kept classes. h: the warp's 256-bin histogram; row: (b, h, query block).
+__device__ void rank_keys_row(const Geo& g, const Ws& w, const uint32_t* keys, uint32_t* h, size_t row,
+                              int lane) {
   const int N = g.N;
   const int n8m = g.n8 + g.nm, nk = g.n8 + g.nm + g.n4;   // the ranking's cuts
   const bool adaptive = g.tau > 0.0f && g.n4max > g.n4;
   const int nkx = g.n8 + g.nm + g.n4max;                    // last rank the adaptive budget may reach
   const uint32_t tau_bits = __float_as_uint(g.tau);       // scores are non-negative: bits order like values
+  // the three cuts of the ranking: n8-th, (n8 + nm)-th and nk-th largest score
+  uint32_t T8 = 0xFFFFFFFFu, Tm = 0xFFFFFFFFu, Tk = 0xFFFFFFFFu;
+  int need8 = 0, needm = 0, needk = 0;
+  if (g.n8 > 0) warp_radix_select(keys, N, g.n8, h, T8, need8);
+  if (g.nm > 0) warp_radix_select(keys, N, n8m, h, Tm, needm);
+  if (nk > 0) warp_radix_select(keys, N, nk, h, Tk, needk);
+  uint32_t Tx = 0xFFFFFFFFu;
+  int needx = 0;
+  if (adaptive) warp_radix_select(keys, N, nkx, h, Tx, needx);
+  int eq8 = 0, eqm = 0, eqk = 0, eqx = 0, c8 = 0, cm = 0, c4 = 0;
+  uint8_t* trow = w.tags + row * N;
+  int16_t* l8 = w.list8 + row * w.n8s;
+  int16_t* lmx = w.listm + row * w.nms;
+  int16_t* l4 = w.list4 + row * w.n4s;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int j0 = 0; j0 < N; j0 += 32) {
+    const int j = j0 + lane;
+    const bool ok = j < N;
+    const uint32_t key = ok ? keys[j] : 0u;
+    // keys equal to a cut value belong above it in block order, as many as the cut needs
+    const uint32_t e8 = __ballot_sync(0xffffffffu, ok && g.n8 > 0 && key == T8);
+    const uint32_t em = __ballot_sync(0xffffffffu, ok && g.nm > 0 && key == Tm);
+    const uint32_t ek = __ballot_sync(0xffffffffu, ok && nk > 0 && key == Tk);
+    const uint32_t ex = __ballot_sync(0xffffffffu, ok && adaptive && key == Tx);
+    const bool in8 = ok && g.n8 > 0 && (key > T8 || (key == T8 && eq8 + __popc(e8 & lt) < need8));
+    const bool in8m = in8 || (ok && g.nm > 0 && (key > Tm || (key == Tm && eqm + __popc(em & lt) < needm)));
+    const bool ink = ok && nk > 0 && (key > Tk || (key == Tk && eqk + __popc(ek & lt) < needk));
+    // adaptive budget: a block ranked after the fixed cut, within the cap, whose score
+    // reaches the threshold joins FP4 (those form a prefix of the ranks, scores being
+    // sorted within the ranking)
+    const bool inx = ok && adaptive && (key > Tx || (key == Tx && eqx + __popc(ex & lt) < needx));
+    const bool rec = inx && !ink && key >= tau_bits;
+    eq8 += __popc(e8);
+    eqm += __popc(em);
+    eqk += __popc(ek);
+    eqx += __popc(ex);
+    const bool inm = in8m && !in8;
+    const bool in4 = (ink && !in8m) || rec;
+    const uint32_t b8 = __ballot_sync(0xffffffffu, in8), bm = __ballot_sync(0xffffffffu, inm),
+                   b4 = __ballot_sync(0xffffffffu, in4);
+    const int p8 = c8 + __popc(b8 & lt), pm = cm + __popc(bm & lt), p4 = c4 + __popc(b4 & lt);
+    if (in8 && p8 < g.n8) l8[p8] = (int16_t)j;
+    if (inm && pm < g.nm) lmx[pm] = (int16_t)j;
+    if (in4 && p4 < g.n4max) l4[p4] = (int16_t)j;
+    c8 += __popc(b8);
+    cm += __popc(bm);
+    c4 += __popc(b4);
+    if (ok) trow[j] = in8 ? 2 : (inm ? 3 : (in4 ? 1 : 0));
+  }
+  for (int p = c4 + lane; p < g.n4max; p += 32) l4[p] = (int16_t)-1;   // no block
+  if (lane == 0 && (c8 != g.n8 || cm != g.nm || c4 < g.n4 || c4 > g.n4max)) set_error(w.err, kErrBadIndex);
+}
+
+// Per-row ranking of the draft scores (one warp per row): the two row softmaxes of the
+// average- and max-pooled logits (in la / lm, R rows of N), their mean as the score, then
+// the shared ranking of the row.
+__device__ void rank_rows(const Geo& g, const Ws& w, float* la, float* lm, uint32_t* hist, int bh, int i0,
+                          int rows, int warp, int lane, int nwarps) {
+  const int N = g.N;
   uint32_t* h = hist + warp * 256;
   for (int r = warp; r < rows; r += nwarps) {
     float* ra = la + r * N;
@@ -116,58 +175,7 @@ __device__ void rank_rows(const Geo& g, const Ws& w, float* la, float* lm, uint3
       if (g.flags & DA2_FLAG_EXPORT_SCORES) w.scores[row * N + j] = sc;
     }
     __syncwarp();
-    const uint32_t* keys = reinterpret_cast<const uint32_t*>(ra);
-    // the three cuts of the ranking: n8-th, (n8 + nm)-th and nk-th largest score
-    uint32_t T8 = 0xFFFFFFFFu, Tm = 0xFFFFFFFFu, Tk = 0xFFFFFFFFu;
-    int need8 = 0, needm = 0, needk = 0;
-    if (g.n8 > 0) warp_radix_select(keys, N, g.n8, h, T8, need8);
-    if (g.nm > 0) warp_radix_select(keys, N, n8m, h, Tm, needm);
-    if (nk > 0) warp_radix_select(keys, N, nk, h, Tk, needk);
-    uint32_t Tx = 0xFFFFFFFFu;
-    int needx = 0;
-    if (adaptive) warp_radix_select(keys, N, nkx, h, Tx, needx);
-    int eq8 = 0, eqm = 0, eqk = 0, eqx = 0, c8 = 0, cm = 0, c4 = 0;
-    uint8_t* trow = w.tags + row * N;
-    int16_t* l8 = w.list8 + row * w.n8s;
-    int16_t* lmx = w.listm + row * w.nms;
-    int16_t* l4 = w.list4 + row * w.n4s;
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int j0 = 0; j0 < N; j0 += 32) {
-      const int j = j0 + lane;
-      const bool ok = j < N;
-      const uint32_t key = ok ? keys[j] : 0u;
-      // keys equal to a cut value belong above it in block order, as many as the cut needs
-      const uint32_t e8 = __ballot_sync(0xffffffffu, ok && g.n8 > 0 && key == T8);
-      const uint32_t em = __ballot_sync(0xffffffffu, ok && g.nm > 0 && key == Tm);
-      const uint32_t ek = __ballot_sync(0xffffffffu, ok && nk > 0 && key == Tk);
-      const uint32_t ex = __ballot_sync(0xffffffffu, ok && adaptive && key == Tx);
-      const bool in8 = ok && g.n8 > 0 && (key > T8 || (key == T8 && eq8 + __popc(e8 & lt) < need8));
-      const bool in8m = in8 || (ok && g.nm > 0 && (key > Tm || (key == Tm && eqm + __popc(em & lt) < needm)));
-      const bool ink = ok && nk > 0 && (key > Tk || (key == Tk && eqk + __popc(ek & lt) < needk));
-      // adaptive budget: a block ranked after the fixed cut, within the cap, whose score
-      // reaches the threshold joins FP4 (those form a prefix of the ranks, scores being
-      // sorted within the ranking)
-      const bool inx = ok && adaptive && (key > Tx || (key == Tx && eqx + __popc(ex & lt) < needx));
-      const bool rec = inx && !ink && key >= tau_bits;
-      eq8 += __popc(e8);
-      eqm += __popc(em);
-      eqk += __popc(ek);
-      eqx += __popc(ex);
-      const bool inm = in8m && !in8;
-      const bool in4 = (ink && !in8m) || rec;
-      const uint32_t b8 = __ballot_sync(0xffffffffu, in8), bm = __ballot_sync(0xffffffffu, inm),
-                     b4 = __ballot_sync(0xffffffffu, in4);
-      const int p8 = c8 + __popc(b8 & lt), pm = cm + __popc(bm & lt), p4 = c4 + __popc(b4 & lt);
-      if (in8 && p8 < g.n8) l8[p8] = (int16_t)j;
-      if (inm && pm < g.nm) lmx[pm] = (int16_t)j;
-      if (in4 && p4 < g.n4max) l4[p4] = (int16_t)j;
-      c8 += __popc(b8);
-      cm += __popc(bm);
-      c4 += __popc(b4);
-      if (ok) trow[j] = in8 ? 2 : (inm ? 3 : (in4 ? 1 : 0));
-    }
-    for (int p = c4 + lane; p < g.n4max; p += 32) l4[p] = (int16_t)-1;   // no block
-    if (lane == 0 && (c8 != g.n8 || cm != g.nm || c4 < g.n4 || c4 > g.n4max)) set_error(w.err, kErrBadIndex);
+    rank_keys_row(g, w, reinterpret_cast<const uint32_t*>(ra), h, row, lane);
   }
 }
 
@@ -451,32 +459,55 @@ size_t logits_tc_smem_bytes(int d) {
   return (size_t)(d / kSplitKC) * 2 * kSplitPart + (size_t)kTcStages * 2 * kSplitPart + 1024 * 4 + 16 * 8;
 }
 
-// Ranking of the draft scores from the logits scratch: 8 query blocks per CTA, one warp each,
-// the same per-row ranking as the other kernels (their two logit rows copied into shared
-// memory first).
-constexpr int kRankRows = 8;
+// Ranking of the draft scores from the logits scratch: one warp per query block, 16 per CTA.
+// Only one N-float row per warp sits in shared memory (the average map's exponentials, then
+// the scores): the maxima and the max map's exponentials are read from the scratch, the
+// latter twice, so that four CTAs (64 warps) fit on an SM. The scores are the same as
+// rank_rows forms (same operations in the same order).
+constexpr int kRankRows = 16;
 __global__ void __launch_bounds__(kRankRows * 32) k_draft_rank(Geo g, Ws w, const float* dlog, int NP) {
   extern __shared__ __align__(16) float rsm[];
   const int N = g.N;
-  float* la = rsm;                                      // [rows][N]
-  float* lm = la + kRankRows * N;                       // [rows][N]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(lm + kRankRows * N);   // [warps][256]
-  const int bh = blockIdx.y, i0 = blockIdx.x * kRankRows;
-  const int rows = min(kRankRows, N - i0);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < rows) {
-    const float* src = dlog + ((size_t)bh * N + i0 + warp) * 2 * NP;
-    for (int j = lane; j < N; j += 32) {
-      la[warp * N + j] = src[j];
-      lm[warp * N + j] = src[NP + j];
-    }
+  const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kRankRows + warp;
+  if (i >= N) return;
+  float* ra = rsm + warp * N;
+  uint32_t* h = reinterpret_cast<uint32_t*>(rsm + kRankRows * N) + warp * 256;
+  const size_t row = (size_t)bh * N + i;
+  const float* la = dlog + row * 2 * NP;
+  const float* lm = la + NP;
+  float mxa = -INFINITY, mxm = -INFINITY;
+  for (int j = lane; j < N; j += 32) { mxa = fmaxf(mxa, la[j]); mxm = fmaxf(mxm, lm[j]); }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, o));
+    mxm = fmaxf(mxm, __shfl_xor_sync(0xffffffffu, mxm, o));
+  }
+  float sa = 0.0f, sm = 0.0f;
+  for (int j = lane; j < N; j += 32) {
+    const float ea = expf(la[j] - mxa), em = expf(lm[j] - mxm);
+    ra[j] = ea;
+    sa += ea;
+    sm += em;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    sm += __shfl_xor_sync(0xffffffffu, sm, o);
+  }
+  const float ia = 1.0f / sa, im = 1.0f / sm;
+  for (int j = lane; j < N; j += 32) {
+    const float em = expf(lm[j] - mxm);
+    const float sc = 0.5f * (ra[j] * ia + em * im);
+    ra[j] = sc;
+    if (g.flags & DA2_FLAG_EXPORT_SCORES) w.scores[row * N + j] = sc;
   }
   __syncwarp();
-  rank_rows(g, w, la, lm, hist, bh, i0, rows, warp, lane, kRankRows);
+  rank_keys_row(g, w, reinterpret_cast<const uint32_t*>(ra), h, row, lane);
 }
 
 size_t rank_smem_bytes(const Geo& g) {
-  return (size_t)2 * kRankRows * g.N * 4 + (size_t)kRankRows * 256 * 4;
+  return (size_t)kRankRows * g.N * 4 + (size_t)kRankRows * 256 * 4;
 }
 
 size_t draft_smem_bytes(const Geo& g, int R) {
