@@ -462,8 +462,8 @@ size_t logits_tc_smem_bytes(int d) {
 // Ranking of the draft scores from the logits scratch: one warp per query block, 16 per CTA.
 // Only one N-float row per warp sits in shared memory (the average map's exponentials, then
 // the scores): the maxima and the max map's exponentials are read from the scratch, the
-// latter twice, so that four CTAs (64 warps) fit on an SM. The scores are the same as
-// rank_rows forms (same operations in the same order).
+// latter twice, so that three CTAs (48 warps; 32 with both rows in shared memory) fit on an
+// SM at N = 630. The scores are the same as rank_rows forms (same operations, same order).
 constexpr int kRankRows = 16;
 __global__ void __launch_bounds__(kRankRows * 32) k_draft_rank(Geo g, Ws w, const float* dlog, int NP) {
   extern __shared__ __align__(16) float rsm[];
