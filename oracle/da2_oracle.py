@@ -10,6 +10,9 @@ Sources (cited by page title and section):
          (arXiv 2505.14708), Abstract.
   [NEWS] News article on DraftAttention (szmaozhuayin.com), method overview steps 1-4 and
          the theoretical-analysis paragraph.
+  [MX]   OCP Microscaling Formats (MX) Specification v1.0, a public standard outside the
+         pages: the MXFP8 element (E4M3) and shared-scale (E8M0, 32 elements) formats used
+         by the block-scaled FP8 variant, which only this oracle implements.
 
 The pages print no equations; where a step is left open the plainest reading is taken
 and listed in the repository's design notes. Every step below is a separate function
@@ -327,6 +330,61 @@ def dequant_v(vd, precision: int) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------------------
+# Block-scaled FP8, oracle only (no CUDA kernel takes this form): MXFP8 as the OCP
+# Microscaling Formats (MX) Specification v1.0 defines it -- 32 consecutive elements along
+# the contraction axis share one E8M0 scale 2^e (e in [-127, 127]) and each element is an
+# E4M3 value of x / 2^e. [DA2] Abstract fixes 8-bit computation for the important blocks,
+# not the scale granularity; this variant puts the scale per 32 elements instead of per
+# block (Q, K) or per head channel (V), so no pre-pass over the head is needed for V.
+# ----------------------------------------------------------------------------------------
+MX_BLOCK = 32
+E4M3_EMAX = 8           # exponent of E4M3's largest normal binade (448 = 1.75 * 2^8)
+
+
+def e8m0_scale_exp(amax) -> np.ndarray:
+    """Shared exponent of an MX block: floor(log2 amax) - 8, clamped to the E8M0 range
+    [-127, 127]; a block whose amax is 0 takes -127 (its elements are then all 0)."""
+    a = np.asarray(amax, dtype=np.float64)
+    safe = np.where(a > 0, a, 1.0)
+    _, fe = np.frexp(safe)                              # safe = m 2^fe, m in [0.5, 1)
+    e = np.where(a > 0, fe - 1 - E4M3_EMAX, -127)
+    return np.clip(e, -127, 127).astype(np.int64)
+
+
+def quantise_mx8(x, axis: int = -1):
+    """MXFP8 of x along `axis` (its length a multiple of 32).
+
+    Returns (codes uint8, same shape as x: E4M3 bytes of x / 2^e, round to nearest even,
+    saturating at +-448; exps int64, shape of x with `axis` divided by 32)."""
+    x = np.moveaxis(np.asarray(x, dtype=np.float64), axis, -1)
+    sh = x.shape
+    xb = x.reshape(sh[:-1] + (sh[-1] // MX_BLOCK, MX_BLOCK))
+    e = e8m0_scale_exp(np.abs(xb).max(axis=-1))
+    codes = e4m3_code(np.ldexp(xb, -e[..., None])).reshape(sh)
+    return np.moveaxis(codes, -1, axis), np.moveaxis(e, -1, axis)
+
+
+def dequant_mx8(codes, exps, axis: int = -1) -> np.ndarray:
+    """fp64 values 2^e * E4M3(code) of an MXFP8 copy blocked along `axis`."""
+    c = np.moveaxis(np.asarray(codes), axis, -1)
+    e = np.moveaxis(np.asarray(exps), axis, -1)
+    sh = c.shape
+    v = e4m3_decode(c).reshape(sh[:-1] + (sh[-1] // MX_BLOCK, MX_BLOCK))
+    v = np.ldexp(v, e[..., None]).reshape(sh)
+    return np.moveaxis(v, -1, axis)
+
+
+def quantise_mx_operands(qp, kp, vp):
+    """MXFP8 copies of the permuted Q, K, V [B,H,N,bs,d]: Q and K blocked along the
+    channels of each token (the Q K^T contraction axis), V along the tokens of each key
+    block per channel (the P V contraction axis). Returns dicts {q8, e} per operand."""
+    q8, qe = quantise_mx8(qp.astype(F32), axis=-1)
+    k8, ke = quantise_mx8(kp.astype(F32), axis=-1)
+    v8, ve = quantise_mx8(vp.astype(F32), axis=-2)
+    return dict(q8=q8, e=qe), dict(q8=k8, e=ke), dict(q8=v8, e=ve)
+
+
+# ----------------------------------------------------------------------------------------
 # Draft maps and ranking ([DA2] Abstract: low-resolution draft attention map from avg- and
 # max-pooled Q/K estimates block importance; a shared ranking gives high precision, low
 # precision or skip under budgets. [DA1] Abstract / [NEWS] step 2: the draft map is the
@@ -439,6 +497,15 @@ def quant_p(p: np.ndarray, precision: int) -> np.ndarray:
     return z.reshape(sh) / E4M3_MAX
 
 
+def quant_p_mx(p: np.ndarray, precision: int) -> np.ndarray:
+    """Probabilities for the block-scaled variant: FP8 as MXFP8 over 32 consecutive keys
+    of a row (fp64 values 2^e E4M3(p / 2^e)); FP4 as `quant_p`."""
+    if precision != 8:
+        return quant_p(p, precision)
+    codes, e = quantise_mx8(p, axis=-1)
+    return dequant_mx8(codes, e, axis=-1)
+
+
 # ----------------------------------------------------------------------------------------
 # Mixed-precision block-sparse attention ([DA2] Abstract: one kernel with precision-
 # specific phases that share data movement, softmax statistics and output accumulation)
@@ -457,13 +524,20 @@ def operands_quantised(qd, kd, vd) -> Operands:
                     {8: dequant_v(vd, 8), 4: dequant_v(vd, 4)})
 
 
+def operands_mx(qd, kd, vd, qmx, kmx, vmx) -> Operands:
+    """8-bit operands from the MXFP8 copies, 4-bit from the NVFP4-style copies."""
+    return Operands({8: dequant_mx8(qmx["q8"], qmx["e"], -1), 4: dequant_qk(qd, 4)},
+                    {8: dequant_mx8(kmx["q8"], kmx["e"], -1), 4: dequant_qk(kd, 4)},
+                    {8: dequant_mx8(vmx["q8"], vmx["e"], -2), 4: dequant_v(vd, 4)})
+
+
 def operands_exact(qp, kp, vp) -> Operands:
     q, k, v = (x.astype(np.float64) for x in (qp, kp, vp))
     return Operands({8: q, 4: q}, {8: k, 4: k}, {8: v, 4: v})
 
 
 def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
-              return_parts=False, blocks=None, listm=None):
+              return_parts=False, blocks=None, listm=None, pquant=quant_p):
     """Block-sparse attention with one online softmax over all phases.
 
     For each (b, h, query block i): the FP8 phase visits list8[i] in ascending block index,
@@ -478,7 +552,8 @@ def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
 
     With return_parts, also returns per (b,h,i) lists of (j, alpha_j, sum p~, sum p~ v)
     for the error decomposition. `blocks`, a list of (b, h, i), restricts the computation
-    to those query blocks (the others stay 0).
+    to those query blocks (the others stay 0). `pquant(p, precision)` quantises the
+    probabilities (`quant_p_mx` for the block-scaled variant).
     """
     B, H, N, bs, d = ops.q[8].shape
     out = np.zeros((B, H, N, bs, d))
@@ -506,7 +581,7 @@ def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
                         alpha = np.where(np.isfinite(m), np.exp(m - np.where(fin, m_new, 0.0)), 0.0)
                         p = np.exp(S - np.where(fin, m_new, 0.0)[:, None])
                         p[~np.isfinite(S)] = 0.0
-                        pq = quant_p(p, pprec) if quantise_p else p
+                        pq = pquant(p, pprec) if quantise_p else p
                         pv = pq @ ops.v[pprec][b, h, j]
                         l = alpha * l + p.sum(axis=1)
                         acc = alpha[:, None] * acc + pv
@@ -630,12 +705,13 @@ def draft_select(prep, mass_correction=True):
     return dict(scores=sc, **r)
 
 
-def run(w, q, k, v, quantised=True, lists=None):
+def run(w, q, k, v, quantised=True, lists=None, fp8="scaled"):
     """Whole hot path. Returns dict with every intermediate and `out` fp64 [B,H,T,d].
 
     `lists` = (list8, list4) or (list8, list4, listm) overrides the oracle's own selection
     (used to compare the attention step on the CUDA path's selection when rankings differ
-    at near-ties).
+    at near-ties). fp8="mx" runs the 8-bit class in the block-scaled MXFP8 form (Q, K, V
+    and P), which only the oracle implements.
     """
     prep = prepare(w, q, k, v)
     g = prep["g"]
@@ -645,10 +721,17 @@ def run(w, q, k, v, quantised=True, lists=None):
     else:
         l8, l4 = lists[0], lists[1]
         lm = lists[2] if len(lists) > 2 else None
-    if quantised:
+    if fp8 not in ("scaled", "mx"):
+        raise ValueError(f"fp8 must be 'scaled' or 'mx', not {fp8!r}")
+    pquant = quant_p
+    if quantised and fp8 == "mx":
+        ops = operands_mx(prep["Q"], prep["K"], prep["V"],
+                          *quantise_mx_operands(prep["qp"], prep["kp"], prep["vp"]))
+        pquant = quant_p_mx
+    elif quantised:
         ops = operands_quantised(prep["Q"], prep["K"], prep["V"])
     else:
         ops = operands_exact(prep["qp"], prep["kp"], prep["vp"])
     o = attention(ops, prep["valid"], l8, l4, g.sm_scale, quantise_p=quantised,
-                  listm=lm if (lm is not None and lm.shape[-1] > 0) else None)
+                  listm=lm if (lm is not None and lm.shape[-1] > 0) else None, pquant=pquant)
     return dict(prep=prep, sel=sel, out_blocks=o, out=inverse_permute(o, g))
