@@ -20,9 +20,43 @@
 
 namespace da2 {
 
+// One pass of an 8-bit radix select within one warp: from the 256-bin histogram of the keys
+// under the current prefix, the digit that holds the remaining-th largest of them and how
+// many keys lie in the digits above it.
+__device__ __forceinline__ void radix_pick(const uint32_t* hist, int remaining, int lane, uint32_t& digit,
+                                           uint32_t& above) {
+  // lane l owns digits 255-8l .. 255-8l-7 (descending)
+  uint32_t c[8];
+  uint32_t s = 0u;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) { c[t] = hist[255 - 8 * lane - t]; s += c[t]; }
+  uint32_t incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t excl = incl - s;
+  const bool mine = excl < (uint32_t)remaining && (uint32_t)remaining <= incl;
+  digit = 0u;
+  above = 0u;
+  if (mine) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (acc + c[t] >= (uint32_t)remaining) { digit = 255u - 8u * lane - t; above = acc; break; }
+      acc += c[t];
+    }
+  }
+  const uint32_t found = __ballot_sync(0xffffffffu, mine);
+  const int src = found ? __ffs(found) - 1 : 0;   // always found when 1 <= remaining <= keys counted
+  digit = __shfl_sync(0xffffffffu, digit, src);
+  above = __shfl_sync(0xffffffffu, above, src);
+}
+
 // k-th largest 32-bit key of `keys[0..n)` (1 <= kth <= n) by an 8-bit radix select within
 // one warp. Returns the key value T and how many of the keys equal to T belong to the top
-// kth (the rest of the top kth are strictly greater than T).
+// kth (the rest of the top kth are strictly greater than T). hist: 256 words.
 __device__ void warp_radix_select(const uint32_t* keys, int n, int kth, uint32_t* hist,
                                   uint32_t& T, int& need) {
   const int lane = threadIdx.x & 31;
@@ -36,32 +70,8 @@ __device__ void warp_radix_select(const uint32_t* keys, int n, int kth, uint32_t
       if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
     }
     __syncwarp();
-    // lane l owns digits 255-8l .. 255-8l-7 (descending)
-    uint32_t c[8];
-    uint32_t s = 0u;
-#pragma unroll
-    for (int t = 0; t < 8; ++t) { c[t] = hist[255 - 8 * lane - t]; s += c[t]; }
-    uint32_t incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const uint32_t excl = incl - s;
-    const bool mine = excl < (uint32_t)remaining && (uint32_t)remaining <= incl;
-    uint32_t digit = 0u, above = 0u;
-    if (mine) {
-      uint32_t acc = excl;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (acc + c[t] >= (uint32_t)remaining) { digit = 255u - 8u * lane - t; above = acc; break; }
-        acc += c[t];
-      }
-    }
-    const uint32_t found = __ballot_sync(0xffffffffu, mine);
-    const int src = found ? __ffs(found) - 1 : 0;   // always found when 1 <= kth <= n
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    above = __shfl_sync(0xffffffffu, above, src);
+    uint32_t digit, above;
+    radix_pick(hist, remaining, lane, digit, above);
     prefix |= digit << shift;
     pmask |= 0xFFu << shift;
     remaining -= (int)above;
@@ -71,11 +81,58 @@ __device__ void warp_radix_select(const uint32_t* keys, int n, int kth, uint32_t
   need = remaining;
 }
 
+// The same select for two ranks at once (1 <= ka, kb <= n): each pass reads the keys once,
+// counting into one histogram while the two cuts' digit prefixes agree and into two once
+// they differ (a key then matches at most one prefix). hist: 512 words.
+__device__ void warp_radix_select2(const uint32_t* keys, int n, int ka, int kb, uint32_t* hist,
+                                   uint32_t& Ta, int& needa, uint32_t& Tb, int& needb) {
+  const int lane = threadIdx.x & 31;
+  uint32_t* ha = hist;
+  uint32_t* hb = hist + 256;
+  uint32_t pa = 0u, pb = 0u, pmask = 0u;
+  int ra = ka, rb = kb;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    const bool same = pa == pb;
+    for (int b = lane; b < (same ? 256 : 512); b += 32) hist[b] = 0u;
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const uint32_t u = keys[j];
+      const uint32_t m = u & pmask, dg = (u >> shift) & 255u;
+      if (m == pa) atomicAdd(&ha[dg], 1u);
+      else if (m == pb) atomicAdd(&hb[dg], 1u);
+    }
+    __syncwarp();
+    uint32_t da, aa, db, ab;
+    radix_pick(ha, ra, lane, da, aa);
+    radix_pick(same ? ha : hb, rb, lane, db, ab);
+    pa |= da << shift;
+    pb |= db << shift;
+    pmask |= 0xFFu << shift;
+    ra -= (int)aa;
+    rb -= (int)ab;
+    __syncwarp();
+  }
+  Ta = pa;
+  needa = ra;
+  Tb = pb;
+  needb = rb;
+}
+
+// The k-th largest for one or two ranks (a rank of 0 is no cut and leaves its outputs).
+__device__ __forceinline__ void radix_cuts(const uint32_t* keys, int n, int ka, int kb, uint32_t* hist,
+                                           uint32_t& Ta, int& needa, uint32_t& Tb, int& needb) {
+  if (ka > 0 && kb > 0) warp_radix_select2(keys, n, ka, kb, hist, Ta, needa, Tb, needb);
+  else if (ka > 0) warp_radix_select(keys, n, ka, hist, Ta, needa);
+  else if (kb > 0) warp_radix_select(keys, n, kb, hist, Tb, needb);
+}
+
+constexpr int kHistWords = 512;   // per warp: the two histograms of warp_radix_select2
+
 constexpr int kDraftThreads = 512, kDraftWarps = kDraftThreads / 32;
 
 // The shared ranking of one score row (one warp; keys = the N scores' bit patterns, which
 // order like the non-negative scores): the radix-select cuts, then tags and the ascending
-// lists of the kept classes. h: the warp's 256-bin histogram; row: (b, h, query block).
+// lists of the kept classes. h: the warp's kHistWords histogram words; row: (b, h, query block).
 __device__ void rank_keys_row(const Geo& g, const Ws& w, const uint32_t* keys, uint32_t* h, size_t row,
                               int lane) {
   const int N = g.N;
@@ -84,14 +141,11 @@ __device__ void rank_keys_row(const Geo& g, const Ws& w, const uint32_t* keys, u
   const int nkx = g.n8 + g.nm + g.n4max;                    // last rank the adaptive budget may reach
   const uint32_t tau_bits = __float_as_uint(g.tau);       // scores are non-negative: bits order like values
   // the three cuts of the ranking: n8-th, (n8 + nm)-th and nk-th largest score
-  uint32_t T8 = 0xFFFFFFFFu, Tm = 0xFFFFFFFFu, Tk = 0xFFFFFFFFu;
-  int need8 = 0, needm = 0, needk = 0;
-  if (g.n8 > 0) warp_radix_select(keys, N, g.n8, h, T8, need8);
-  if (g.nm > 0) warp_radix_select(keys, N, n8m, h, Tm, needm);
-  if (nk > 0) warp_radix_select(keys, N, nk, h, Tk, needk);
-  uint32_t Tx = 0xFFFFFFFFu;
-  int needx = 0;
-  if (adaptive) warp_radix_select(keys, N, nkx, h, Tx, needx);
+  // (and the adaptive cap's nkx-th), selected two at a time
+  uint32_t T8 = 0xFFFFFFFFu, Tm = 0xFFFFFFFFu, Tk = 0xFFFFFFFFu, Tx = 0xFFFFFFFFu;
+  int need8 = 0, needm = 0, needk = 0, needx = 0;
+  radix_cuts(keys, N, g.n8, nk, h, T8, need8, Tk, needk);
+  radix_cuts(keys, N, g.nm > 0 ? n8m : 0, adaptive ? nkx : 0, h, Tm, needm, Tx, needx);
   int eq8 = 0, eqm = 0, eqk = 0, eqx = 0, c8 = 0, cm = 0, c4 = 0;
   uint8_t* trow = w.tags + row * N;
   int16_t* l8 = w.list8 + row * w.n8s;
@@ -142,7 +196,7 @@ __device__ void rank_keys_row(const Geo& g, const Ws& w, const uint32_t* keys, u
 __device__ void rank_rows(const Geo& g, const Ws& w, float* la, float* lm, uint32_t* hist, int bh, int i0,
                           int rows, int warp, int lane, int nwarps) {
   const int N = g.N;
-  uint32_t* h = hist + warp * 256;
+  uint32_t* h = hist + warp * kHistWords;
   for (int r = warp; r < rows; r += nwarps) {
     float* ra = la + r * N;
     float* rm = lm + r * N;
@@ -188,7 +242,7 @@ __global__ void __launch_bounds__(kDraftThreads) k_draft_select(Geo g, Ws w, int
   float* qm = qa + R * D;          // [R][D]
   float* la = qm + R * D;          // [R][N]  avg logits, later the score
   float* lm = la + R * N;          // [R][N]  max logits
-  uint32_t* hist = reinterpret_cast<uint32_t*>(lm + R * N);  // [warps][256]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(lm + R * N);  // [warps][kHistWords]
   const int bh = blockIdx.y, i0 = blockIdx.x * R;
   const int rows = min(R, N - i0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -459,11 +513,21 @@ size_t logits_tc_smem_bytes(int d) {
   return (size_t)(d / kSplitKC) * 2 * kSplitPart + (size_t)kTcStages * 2 * kSplitPart + 1024 * 4 + 16 * 8;
 }
 
+// e^t for t <= 0 (a logit minus its row max) as 2^(t log2 e) on the special-function unit
+// (ex2.approx.ftz.f32): two instructions instead of the accurate expf's range reduction.
+// Its relative error, a few units in the last place, stays far inside the ranking's
+// tolerance; results below 2^-126 flush to zero.
+__device__ __forceinline__ float exp_sfu(float t) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(t * 1.4426950408889634f));
+  return y;
+}
+
 // Ranking of the draft scores from the logits scratch: one warp per query block, 16 per CTA.
 // Only one N-float row per warp sits in shared memory (the average map's exponentials, then
 // the scores): the maxima and the max map's exponentials are read from the scratch, the
-// latter twice, so that three CTAs (48 warps; 32 with both rows in shared memory) fit on an
-// SM at N = 630. The scores are the same as rank_rows forms (same operations, same order).
+// latter twice, so that three CTAs (48 warps) fit on an SM at N = 630. The scores are
+// formed as in rank_rows except for the exponentials, taken here by exp_sfu.
 constexpr int kRankRows = 16;
 __global__ void __launch_bounds__(kRankRows * 32) k_draft_rank(Geo g, Ws w, const float* dlog, int NP) {
   extern __shared__ __align__(16) float rsm[];
@@ -472,7 +536,7 @@ __global__ void __launch_bounds__(kRankRows * 32) k_draft_rank(Geo g, Ws w, cons
   const int i = blockIdx.x * kRankRows + warp;
   if (i >= N) return;
   float* ra = rsm + warp * N;
-  uint32_t* h = reinterpret_cast<uint32_t*>(rsm + kRankRows * N) + warp * 256;
+  uint32_t* h = reinterpret_cast<uint32_t*>(rsm + kRankRows * N) + warp * kHistWords;
   const size_t row = (size_t)bh * N + i;
   const float* la = dlog + row * 2 * NP;
   const float* lm = la + NP;
@@ -485,7 +549,7 @@ __global__ void __launch_bounds__(kRankRows * 32) k_draft_rank(Geo g, Ws w, cons
   }
   float sa = 0.0f, sm = 0.0f;
   for (int j = lane; j < N; j += 32) {
-    const float ea = expf(la[j] - mxa), em = expf(lm[j] - mxm);
+    const float ea = exp_sfu(la[j] - mxa), em = exp_sfu(lm[j] - mxm);
     ra[j] = ea;
     sa += ea;
     sm += em;
@@ -497,7 +561,7 @@ __global__ void __launch_bounds__(kRankRows * 32) k_draft_rank(Geo g, Ws w, cons
   }
   const float ia = 1.0f / sa, im = 1.0f / sm;
   for (int j = lane; j < N; j += 32) {
-    const float em = expf(lm[j] - mxm);
+    const float em = exp_sfu(lm[j] - mxm);
     const float sc = 0.5f * (ra[j] * ia + em * im);
     ra[j] = sc;
     if (g.flags & DA2_FLAG_EXPORT_SCORES) w.scores[row * N + j] = sc;
@@ -507,11 +571,11 @@ __global__ void __launch_bounds__(kRankRows * 32) k_draft_rank(Geo g, Ws w, cons
 }
 
 size_t rank_smem_bytes(const Geo& g) {
-  return (size_t)kRankRows * g.N * 4 + (size_t)kRankRows * 256 * 4;
+  return (size_t)kRankRows * g.N * 4 + (size_t)kRankRows * kHistWords * 4;
 }
 
 size_t draft_smem_bytes(const Geo& g, int R) {
-  return (size_t)(2 * R * g.d + 2 * R * g.N) * 4 + kDraftWarps * 256 * 4;
+  return (size_t)(2 * R * g.d + 2 * R * g.N) * 4 + kDraftWarps * kHistWords * 4;
 }
 
 int draft_rows_per_cta(const Geo& g) {
