@@ -133,11 +133,13 @@ constexpr int kDraftThreads = 512, kDraftWarps = kDraftThreads / 32;
 // The shared ranking of one score row (one warp; keys = the N scores' bit patterns, which
 // order like the non-negative scores): the radix-select cuts, then tags and the ascending
 // lists of the kept classes. h: the warp's kHistWords histogram words; row: (b, h, query block).
-__device__ void rank_keys_row(const Geo& g, const Ws& w, const uint32_t* keys, uint32_t* h, size_t row,
-                              int lane) {
+// MIX: a mixed class (nm > 0); ADAPT: the adaptive FP4 budget (tau > 0, n4max > n4). Without
+// them the row needs neither their cuts nor their per-key tests.
+template <bool MIX, bool ADAPT>
+__device__ __forceinline__ void rank_keys_row_t(const Geo& g, const Ws& w, const uint32_t* keys, uint32_t* h, size_t row,
+                                int lane) {
   const int N = g.N;
   const int n8m = g.n8 + g.nm, nk = g.n8 + g.nm + g.n4;   // the ranking's cuts
-  const bool adaptive = g.tau > 0.0f && g.n4max > g.n4;
   const int nkx = g.n8 + g.nm + g.n4max;                    // last rank the adaptive budget may reach
   const uint32_t tau_bits = __float_as_uint(g.tau);       // scores are non-negative: bits order like values
   // the three cuts of the ranking: n8-th, (n8 + nm)-th and nk-th largest score
@@ -145,7 +147,7 @@ __device__ void rank_keys_row(const Geo& g, const Ws& w, const uint32_t* keys, u
   uint32_t T8 = 0xFFFFFFFFu, Tm = 0xFFFFFFFFu, Tk = 0xFFFFFFFFu, Tx = 0xFFFFFFFFu;
   int need8 = 0, needm = 0, needk = 0, needx = 0;
   radix_cuts(keys, N, g.n8, nk, h, T8, need8, Tk, needk);
-  radix_cuts(keys, N, g.nm > 0 ? n8m : 0, adaptive ? nkx : 0, h, Tm, needm, Tx, needx);
+  if (MIX || ADAPT) radix_cuts(keys, N, MIX ? n8m : 0, ADAPT ? nkx : 0, h, Tm, needm, Tx, needx);
   int eq8 = 0, eqm = 0, eqk = 0, eqx = 0, c8 = 0, cm = 0, c4 = 0;
   uint8_t* trow = w.tags + row * N;
   int16_t* l8 = w.list8 + row * w.n8s;
@@ -158,36 +160,51 @@ __device__ void rank_keys_row(const Geo& g, const Ws& w, const uint32_t* keys, u
     const uint32_t key = ok ? keys[j] : 0u;
     // keys equal to a cut value belong above it in block order, as many as the cut needs
     const uint32_t e8 = __ballot_sync(0xffffffffu, ok && g.n8 > 0 && key == T8);
-    const uint32_t em = __ballot_sync(0xffffffffu, ok && g.nm > 0 && key == Tm);
+    const uint32_t em = MIX ? __ballot_sync(0xffffffffu, ok && key == Tm) : 0u;
     const uint32_t ek = __ballot_sync(0xffffffffu, ok && nk > 0 && key == Tk);
-    const uint32_t ex = __ballot_sync(0xffffffffu, ok && adaptive && key == Tx);
+    const uint32_t ex = ADAPT ? __ballot_sync(0xffffffffu, ok && key == Tx) : 0u;
     const bool in8 = ok && g.n8 > 0 && (key > T8 || (key == T8 && eq8 + __popc(e8 & lt) < need8));
-    const bool in8m = in8 || (ok && g.nm > 0 && (key > Tm || (key == Tm && eqm + __popc(em & lt) < needm)));
+    const bool in8m = in8 || (MIX && ok && (key > Tm || (key == Tm && eqm + __popc(em & lt) < needm)));
     const bool ink = ok && nk > 0 && (key > Tk || (key == Tk && eqk + __popc(ek & lt) < needk));
     // adaptive budget: a block ranked after the fixed cut, within the cap, whose score
     // reaches the threshold joins FP4 (those form a prefix of the ranks, scores being
     // sorted within the ranking)
-    const bool inx = ok && adaptive && (key > Tx || (key == Tx && eqx + __popc(ex & lt) < needx));
+    const bool inx = ADAPT && ok && (key > Tx || (key == Tx && eqx + __popc(ex & lt) < needx));
     const bool rec = inx && !ink && key >= tau_bits;
     eq8 += __popc(e8);
-    eqm += __popc(em);
     eqk += __popc(ek);
-    eqx += __popc(ex);
+    if (MIX) eqm += __popc(em);
+    if (ADAPT) eqx += __popc(ex);
     const bool inm = in8m && !in8;
     const bool in4 = (ink && !in8m) || rec;
-    const uint32_t b8 = __ballot_sync(0xffffffffu, in8), bm = __ballot_sync(0xffffffffu, inm),
-                   b4 = __ballot_sync(0xffffffffu, in4);
-    const int p8 = c8 + __popc(b8 & lt), pm = cm + __popc(bm & lt), p4 = c4 + __popc(b4 & lt);
+    const uint32_t b8 = __ballot_sync(0xffffffffu, in8), b4 = __ballot_sync(0xffffffffu, in4);
+    const uint32_t bm = MIX ? __ballot_sync(0xffffffffu, inm) : 0u;
+    const int p8 = c8 + __popc(b8 & lt), p4 = c4 + __popc(b4 & lt);
     if (in8 && p8 < g.n8) l8[p8] = (int16_t)j;
-    if (inm && pm < g.nm) lmx[pm] = (int16_t)j;
     if (in4 && p4 < g.n4max) l4[p4] = (int16_t)j;
+    if (MIX) {
+      const int pm = cm + __popc(bm & lt);
+      if (inm && pm < g.nm) lmx[pm] = (int16_t)j;
+      cm += __popc(bm);
+    }
     c8 += __popc(b8);
-    cm += __popc(bm);
     c4 += __popc(b4);
     if (ok) trow[j] = in8 ? 2 : (inm ? 3 : (in4 ? 1 : 0));
   }
   for (int p = c4 + lane; p < g.n4max; p += 32) l4[p] = (int16_t)-1;   // no block
   if (lane == 0 && (c8 != g.n8 || cm != g.nm || c4 < g.n4 || c4 > g.n4max)) set_error(w.err, kErrBadIndex);
+}
+
+__device__ __forceinline__ void rank_keys_row(const Geo& g, const Ws& w, const uint32_t* keys, uint32_t* h,
+                                              size_t row, int lane) {
+  const bool mix = g.nm > 0, adapt = g.tau > 0.0f && g.n4max > g.n4;
+  if (mix) {
+    if (adapt) rank_keys_row_t<true, true>(g, w, keys, h, row, lane);
+    else rank_keys_row_t<true, false>(g, w, keys, h, row, lane);
+  } else {
+    if (adapt) rank_keys_row_t<false, true>(g, w, keys, h, row, lane);
+    else rank_keys_row_t<false, false>(g, w, keys, h, row, lane);
+  }
 }
 
 // Per-row ranking of the draft scores (one warp per row): the two row softmaxes of the
