@@ -14,6 +14,9 @@ Sources (cited by page title and section):
          pages: the MXFP8 element (E4M3) and shared-scale (E8M0, 32 elements) formats used
          by the block-scaled FP8 variant, which only this oracle implements.
 
+Only this oracle implements the bf16 top tier either: a class above FP8 whose blocks run
+both products on the bf16 input values with P rounded to bf16 (`bf16_round`).
+
 The pages print no equations; where a step is left open the plainest reading is taken
 and listed in the repository's design notes. Every step below is a separate function
 returning its own arrays so that each can be compared with the CUDA path on its own.
@@ -37,7 +40,7 @@ import numpy as np
 F32 = np.float32
 E4M3_MAX = 448.0        # largest finite E4M3 value (OCP FP8, bias 7, no infinities)
 E2M1_MAX = 6.0          # largest E2M1 value
-TAG_SKIP, TAG_FP4, TAG_FP8, TAG_MIX = 0, 1, 2, 3
+TAG_SKIP, TAG_FP4, TAG_FP8, TAG_MIX, TAG_BF16 = 0, 1, 2, 3, 4
 
 
 # ----------------------------------------------------------------------------------------
@@ -65,6 +68,7 @@ class Geometry:
     nm: int = 0   # mixed blocks per query block (E4M3 scores, E2M1 P V)
     n4max: int = 0  # FP4 list length with the adaptive budget (n4 when it is off)
     tau: float = 0.0  # adaptive budget threshold on the draft score (0: off)
+    n16: int = 0  # bf16 blocks per query block (the tier above FP8; oracle only)
 
 
 def budget_counts(N: int, pct_fp8: int, pct_fp4: int) -> tuple[int, int]:
@@ -94,17 +98,32 @@ def budget_counts3(N: int, pct_fp8: int, pct_mix: int, pct_fp4: int) -> tuple[in
     return c8, c8m - c8, ck - c8m
 
 
+def budget_counts_tiers(N: int, pct_bf16: int, pct_fp8: int, pct_mix: int,
+                       pct_fp4: int) -> tuple[int, int, int, int]:
+    """Blocks kept at bf16, FP8, mixed and FP4 per query block: the four classes take the
+    ranking's top blocks in that order, each cumulative cut rounded half up as in
+    `budget_counts` (with pct_bf16 = 0 the last three are those of `budget_counts3`).
+
+    [DA2] Abstract: higher precision for the more important blocks, lower precision for
+    the rest. Reading: bf16 (the input precision) is the highest, so its class comes first.
+    """
+    c16 = (pct_bf16 * N + 50) // 100
+    n8, nm, n4 = budget_counts3(N, pct_bf16 + pct_fp8, pct_mix, pct_fp4)
+    return c16, n8 - c16, nm, n4
+
+
 def geometry(w) -> Geometry:
     ny, nx = -(-w.Hf // w.ph), -(-w.Wf // w.pw)
     N = w.F * ny * nx
     bs = w.ph * w.pw
     pm = getattr(w, "pct_mix", 0)
-    n8, nm, n4 = budget_counts3(N, w.pct_fp8, pm, w.pct_fp4)
+    p16 = getattr(w, "pct_bf16", 0)
+    n16, n8, nm, n4 = budget_counts_tiers(N, p16, w.pct_fp8, pm, w.pct_fp4)
     tau = float(np.float32(getattr(w, "adapt_tau", 0.0)))      # a configuration value in fp32
-    n4max = budget_counts3(N, w.pct_fp8, pm, w.pct_fp4_max)[2] if tau > 0 else n4
+    n4max = budget_counts_tiers(N, p16, w.pct_fp8, pm, w.pct_fp4_max)[3] if tau > 0 else n4
     sm = getattr(w, "sm_scale", 0.0) or 1.0 / math.sqrt(w.d)
     return Geometry(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, ny, nx, N, bs,
-                    w.F * w.Hf * w.Wf, N * bs, n8, n4, sm, nm, n4max, tau)
+                    w.F * w.Hf * w.Wf, N * bs, n8, n4, sm, nm, n4max, tau, n16)
 
 
 def token_block_slot(g: Geometry):
@@ -216,6 +235,19 @@ def e2m1_round(y) -> np.ndarray:
     a = np.abs(y)
     quantum = np.where(a < 2.0, 0.5, np.where(a < 4.0, 1.0, 2.0))
     r = np.minimum(np.rint(a / quantum) * quantum, E2M1_MAX)
+    return np.copysign(r, y)
+
+
+def bf16_round(y) -> np.ndarray:
+    """Nearest bfloat16 value (fp64), ties to even mantissa: 8 significant bits (1 implicit
+    + 7 stored), normal exponents down to 2^-126 and subnormal steps of 2^-133 below; values
+    that round past the largest finite bf16 (about 3.39e38) become infinite."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    _, e = np.frexp(a)                                  # a = m 2^e, m in [0.5, 1)
+    quantum = np.where(a >= 2.0 ** -126, np.ldexp(1.0, e - 8), 2.0 ** -133)
+    r = np.rint(a / quantum) * quantum
+    r = np.where(r > (2.0 - 2.0 ** -7) * 2.0 ** 127, np.inf, r)
     return np.copysign(r, y)
 
 
@@ -409,12 +441,14 @@ def draft_scores(qavg, kavg, qmax, kmax, counts, sm_scale, mass_correction=True)
     return 0.5 * (one(qavg, kavg) + one(qmax, kmax))
 
 
-def rank_classes(scores, n8: int, nm: int, n4: int):
-    """Shared ranking of each row into four classes: order (score desc, block index asc);
-    the first n8 blocks are FP8, the next nm mixed, the next n4 FP4, the rest skipped.
+def rank_classes(scores, n8: int, nm: int, n4: int, n16: int = 0):
+    """Shared ranking of each row into the precision classes: order (score desc, block
+    index asc); the first n16 blocks are bf16, the next n8 FP8, the next nm mixed, the next
+    n4 FP4, the rest skipped.
 
-    Returns tags uint8 [..., N, N] (0 skip, 1 FP4, 2 FP8, 3 mixed) and the ascending block
-    lists of each kept class: list8 [..., N, n8], listm [..., N, nm], list4 [..., N, n4].
+    Returns tags uint8 [..., N, N] (0 skip, 1 FP4, 2 FP8, 3 mixed, 4 bf16) and the ascending
+    block lists of each kept class: list16 [..., N, n16], list8 [..., N, n8], listm
+    [..., N, nm], list4 [..., N, n4].
     """
     sc = np.asarray(scores)
     lead = sc.shape[:-1]
@@ -422,7 +456,8 @@ def rank_classes(scores, n8: int, nm: int, n4: int):
     flat = sc.reshape(-1, N)
     j = np.arange(N)
     tags = np.zeros(flat.shape, dtype=np.uint8)
-    cuts = ((TAG_FP8, 0, n8), (TAG_MIX, n8, n8 + nm), (TAG_FP4, n8 + nm, n8 + nm + n4))
+    c8, c8m = n16 + n8, n16 + n8 + nm
+    cuts = ((TAG_BF16, 0, n16), (TAG_FP8, n16, c8), (TAG_MIX, c8, c8m), (TAG_FP4, c8m, c8m + n4))
     lists = {t: np.zeros((flat.shape[0], b - a), dtype=np.int64) for t, a, b in cuts}
     for r in range(flat.shape[0]):
         order = np.lexsort((j, -flat[r]))
@@ -430,12 +465,13 @@ def rank_classes(scores, n8: int, nm: int, n4: int):
             tags[r, order[a:b]] = t
             lists[t][r] = np.sort(order[a:b])
     return dict(tags=tags.reshape(lead + (N,)),
+                list16=lists[TAG_BF16].reshape(lead + (n16,)),
                 list8=lists[TAG_FP8].reshape(lead + (n8,)),
                 listm=lists[TAG_MIX].reshape(lead + (nm,)),
                 list4=lists[TAG_FP4].reshape(lead + (n4,)))
 
 
-def rank_adaptive(scores, n8: int, nm: int, n4: int, n4max: int, tau: float):
+def rank_adaptive(scores, n8: int, nm: int, n4: int, n4max: int, tau: float, n16: int = 0):
     """The shared ranking with an error-bound-driven FP4 budget per row.
 
     [DA2] Abstract: the analysis separates the sparsification error from the
@@ -449,7 +485,7 @@ def rank_adaptive(scores, n8: int, nm: int, n4: int, n4max: int, tau: float):
     the row holds n4max FP4 blocks. list4 keeps ascending block order and is padded to n4max
     entries with -1 (no block); count4 holds each row's FP4 count.
     """
-    r = rank_classes(scores, n8, nm, n4)
+    r = rank_classes(scores, n8, nm, n4, n16)
     sc = np.asarray(scores)
     lead = sc.shape[:-1]
     N = sc.shape[-1]
@@ -458,7 +494,7 @@ def rank_adaptive(scores, n8: int, nm: int, n4: int, n4max: int, tau: float):
     l4 = np.full((flat.shape[0], n4max), -1, dtype=np.int64)
     cnt = np.zeros(flat.shape[0], dtype=np.int64)
     j = np.arange(N)
-    ck, ckmax = n8 + nm + n4, min(n8 + nm + n4max, N)
+    ck, ckmax = n16 + n8 + nm + n4, min(n16 + n8 + nm + n4max, N)
     base4 = r["list4"].reshape(flat.shape[0], n4)
     for row in range(flat.shape[0]):
         order = np.lexsort((j, -flat[row]))
@@ -469,8 +505,8 @@ def rank_adaptive(scores, n8: int, nm: int, n4: int, n4max: int, tau: float):
         kept = np.sort(np.concatenate([base4[row], np.array(extra, dtype=np.int64)]))
         l4[row, :len(kept)] = kept
         cnt[row] = len(kept)
-    return dict(tags=tags.reshape(lead + (N,)), list8=r["list8"], listm=r["listm"],
-                list4=l4.reshape(lead + (n4max,)), count4=cnt.reshape(lead))
+    return dict(tags=tags.reshape(lead + (N,)), list16=r["list16"], list8=r["list8"],
+                listm=r["listm"], list4=l4.reshape(lead + (n4max,)), count4=cnt.reshape(lead))
 
 
 def rank(scores, n8: int, n4: int):
@@ -484,8 +520,11 @@ def rank(scores, n8: int, n4: int):
 # precision). p = exp(S - m) <= 1 with m the running row max.
 # ----------------------------------------------------------------------------------------
 def quant_p(p: np.ndarray, precision: int) -> np.ndarray:
-    """Quantised probabilities (fp64). FP8: E4M3(448 p)/448. FP4: y = 448 p, groups of 16
-    consecutive keys, sigma = E4M3(amax16/6), value sigma*E2M1(y/sigma)/448."""
+    """Quantised probabilities (fp64). bf16 (precision 16): bf16(p). FP8: E4M3(448 p)/448.
+    FP4: y = 448 p, groups of 16 consecutive keys, sigma = E4M3(amax16/6), value
+    sigma*E2M1(y/sigma)/448."""
+    if precision == 16:
+        return bf16_round(p)
     y = p * E4M3_MAX
     if precision == 8:
         return e4m3_round(y) / E4M3_MAX
@@ -512,7 +551,8 @@ def quant_p_mx(p: np.ndarray, precision: int) -> np.ndarray:
 # ----------------------------------------------------------------------------------------
 @dataclass
 class Operands:
-    """fp64 operand values per precision: q8/q4/k8/k4/v8/v4 [B,H,N,bs,d]."""
+    """fp64 operand values per precision: q8/q4/k8/k4/v8/v4 [B,H,N,bs,d], and q16/k16/v16
+    (the bf16 input values) where the bf16 tier runs."""
     q: dict
     k: dict
     v: dict
@@ -533,14 +573,23 @@ def operands_mx(qd, kd, vd, qmx, kmx, vmx) -> Operands:
 
 def operands_exact(qp, kp, vp) -> Operands:
     q, k, v = (x.astype(np.float64) for x in (qp, kp, vp))
-    return Operands({8: q, 4: q}, {8: k, 4: k}, {8: v, 4: v})
+    return Operands({16: q, 8: q, 4: q}, {16: k, 8: k, 4: k}, {16: v, 8: v, 4: v})
+
+
+def with_bf16(ops: Operands, qp, kp, vp) -> Operands:
+    """`ops` plus the bf16 tier's operands: the permuted input values themselves (the
+    inputs are bf16, so the tier needs no quantiser)."""
+    return Operands({**ops.q, 16: qp.astype(np.float64)}, {**ops.k, 16: kp.astype(np.float64)},
+                    {**ops.v, 16: vp.astype(np.float64)})
 
 
 def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
-              return_parts=False, blocks=None, listm=None, pquant=quant_p):
+              return_parts=False, blocks=None, listm=None, pquant=quant_p, list16=None):
     """Block-sparse attention with one online softmax over all phases.
 
-    For each (b, h, query block i): the FP8 phase visits list8[i] in ascending block index,
+    For each (b, h, query block i): the bf16 phase (when list16 is given) visits list16[i]
+    (bf16 operands, P rounded to bf16), then the FP8 phase visits list8[i] in ascending
+    block index,
     then the mixed phase visits listm[i] (scores from the E4M3 copies of Q and K, P
     quantised as for FP4 and multiplied with the E2M1 copy of V), then the FP4 phase visits
     list4[i]; each visited block j updates the running row max
@@ -565,7 +614,8 @@ def attention(ops: Operands, valid, list8, list4, sm_scale, quantise_p=True,
                 l = np.zeros(bs)
                 acc = np.zeros((bs, d))
                 rec = []
-                phases = [(8, 8, list8[b, h, i])]
+                phases = [(16, 16, list16[b, h, i])] if list16 is not None else []
+                phases.append((8, 8, list8[b, h, i]))
                 if listm is not None:
                     phases.append((8, 4, listm[b, h, i]))
                 phases.append((4, 4, list4[b, h, i]))
@@ -699,9 +749,9 @@ def draft_select(prep, mass_correction=True):
     sc = draft_scores(prep["qavg"], prep["kavg"], prep["qmax"], prep["kmax"],
                       prep["counts"], g.sm_scale, mass_correction)
     if g.tau > 0:
-        r = rank_adaptive(sc, g.n8, g.nm, g.n4, g.n4max, g.tau)
+        r = rank_adaptive(sc, g.n8, g.nm, g.n4, g.n4max, g.tau, g.n16)
     else:
-        r = rank_classes(sc, g.n8, g.nm, g.n4)
+        r = rank_classes(sc, g.n8, g.nm, g.n4, g.n16)
     return dict(scores=sc, **r)
 
 
@@ -711,7 +761,8 @@ def run(w, q, k, v, quantised=True, lists=None, fp8="scaled"):
     `lists` = (list8, list4) or (list8, list4, listm) overrides the oracle's own selection
     (used to compare the attention step on the CUDA path's selection when rankings differ
     at near-ties). fp8="mx" runs the 8-bit class in the block-scaled MXFP8 form (Q, K, V
-    and P), which only the oracle implements.
+    and P), which only the oracle implements; so does the bf16 tier (a workload with
+    pct_bf16 > 0).
     """
     prep = prepare(w, q, k, v)
     g = prep["g"]
@@ -721,6 +772,7 @@ def run(w, q, k, v, quantised=True, lists=None, fp8="scaled"):
     else:
         l8, l4 = lists[0], lists[1]
         lm = lists[2] if len(lists) > 2 else None
+    l16 = sel["list16"] if g.n16 > 0 else None
     if fp8 not in ("scaled", "mx"):
         raise ValueError(f"fp8 must be 'scaled' or 'mx', not {fp8!r}")
     pquant = quant_p
@@ -732,6 +784,9 @@ def run(w, q, k, v, quantised=True, lists=None, fp8="scaled"):
         ops = operands_quantised(prep["Q"], prep["K"], prep["V"])
     else:
         ops = operands_exact(prep["qp"], prep["kp"], prep["vp"])
+    if l16 is not None:
+        ops = with_bf16(ops, prep["qp"], prep["kp"], prep["vp"])
     o = attention(ops, prep["valid"], l8, l4, g.sm_scale, quantise_p=quantised,
-                  listm=lm if (lm is not None and lm.shape[-1] > 0) else None, pquant=pquant)
+                  listm=lm if (lm is not None and lm.shape[-1] > 0) else None, pquant=pquant,
+                  list16=l16)
     return dict(prep=prep, sel=sel, out_blocks=o, out=inverse_permute(o, g))

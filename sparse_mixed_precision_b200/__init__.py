@@ -121,7 +121,12 @@ EXPORTED = ("da2_workspace_size", "da2_workspace_views", "da2_prepare", "da2_dra
 
 
 def config(w, flags: int = 0, sm_scale: float = 0.0) -> Config:
-    """da2_config of a synth.Workload (or any object with the same fields)."""
+    """da2_config of a synth.Workload (or any object with the same fields).
+
+    The library has no bf16 tier (a workload with pct_bf16 > 0): such a workload is refused
+    here rather than run without its bf16 blocks."""
+    if int(getattr(w, "pct_bf16", 0)) != 0:
+        raise ValueError("the library has no bf16 tier: pct_bf16 must be 0")
     return Config(w.B, w.H, w.d, w.F, w.Hf, w.Wf, w.ph, w.pw, w.pct_fp8, w.pct_fp4,
                   float(sm_scale), int(flags), int(getattr(w, "pct_mix", 0)),
                   float(getattr(w, "adapt_tau", 0.0)), int(getattr(w, "pct_fp4_max", 0)))

@@ -43,6 +43,7 @@ class Workload:
     pct_mix: int = 0     # percent of KV blocks with E4M3 scores and E2M1 P V (between FP8 and FP4)
     adapt_tau: float = 0.0   # > 0: skipped blocks with draft score >= adapt_tau join FP4 ...
     pct_fp4_max: int = 0     # ... up to this FP4 budget (percent)
+    pct_bf16: int = 0        # percent of KV blocks in the bf16 tier above FP8 (the oracle only)
 
     @property
     def T(self) -> int:

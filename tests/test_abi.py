@@ -206,3 +206,11 @@ def test_check_selection_rejects_bad_arguments_without_touching_the_device():
     assert L.da2_check_selection(ctypes.byref(cfg), None, n, None) == 1
     assert L.da2_check_selection(ctypes.byref(cfg), ctypes.c_void_p(0x1008), n, None) == 3
     assert L.da2_check_selection(ctypes.byref(cfg), ctypes.c_void_p(0x100000), n - 1, None) == 4
+
+
+def test_binding_refuses_a_bf16_budget():
+    # the bf16 tier exists in the oracle only: a configuration with bf16 blocks is refused
+    # instead of being run as if those blocks were skipped
+    with pytest.raises(ValueError, match="bf16"):
+        da2.config(scaled(WORKLOADS["tiny"], pct_bf16=5))
+    assert da2.config(scaled(WORKLOADS["tiny"], pct_bf16=0)).pct_fp8 == WORKLOADS["tiny"].pct_fp8
