@@ -27,8 +27,8 @@ order, then an IEEE fp32 divide), the operand scales and the operand quantisers 
 fp32 multiplies/divides, then round-to-nearest-even onto the E4M3 / E2M1 grids).
 
 Parity pins: every function is pinned by `tests/test_oracle_*.py` against closed forms,
-library routines or brute force; the error-decomposition formula itself is not printed
-on the pages (parity unpinned, see `error_decomposition`).
+library routines or brute force. The error-decomposition formula is a reading (the pages
+print none); its terms are pinned by torch and by closed forms, see `error_decomposition`.
 """
 from __future__ import annotations
 
@@ -660,8 +660,10 @@ def dense_attention(q, k, v, sm_scale, key_mask=None):
 
 # ----------------------------------------------------------------------------------------
 # Error decomposition ([DA2] Abstract: the analysis separates the sparsification error
-# from an attention-weighted quantisation error). The formula is not printed on the pages:
-# parity unpinned. Reading: per query row, with O dense, O_S the exact attention over the
+# from an attention-weighted quantisation error). The formula is not printed on the pages;
+# the reading below is pinned term by term (the skipped mass and E_sp by torch's softmax
+# and SDPA, E_q by a closed form for constant scores and by the bound it must satisfy).
+# Reading: per query row, with O dense, O_S the exact attention over the
 # kept blocks, O~ the mixed result,
 #   E_sp = ||O_S - O|| = m_skip ||o_skip - O_S||   (m_skip: softmax mass of skipped blocks)
 #   E_q  = sum_b w_b ||o~_b - o_b|| + sum_b |w~_b - w_b| ||o~_b||
