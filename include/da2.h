@@ -45,7 +45,8 @@
  *    enqueued; a failed CUDA call or launch returns DA2_ERR_CUDA, and da2_last_cuda_error
  *    then gives its cudaError_t.
  *  - Supported: d in {64, 128}; any window with bs = ph*pw in {32, 64, 128}; N <= 4096;
- *    0 <= pct_fp8, pct_mix, pct_fp4 and pct_fp8 + pct_mix + pct_fp4 <= 100. Tensor pointers must be 16-byte
+ *    B*H <= 65535 (DA2_ERR_UNSUPPORTED otherwise); 0 <= pct_fp8, pct_mix, pct_fp4 and
+ *    pct_fp8 + pct_mix + pct_fp4 <= 100 (DA2_ERR_INVALID_ARG otherwise). Tensor pointers must be 16-byte
  *    aligned and the workspace 256-byte aligned (DA2_ERR_ALIGNMENT otherwise).
  */
 #ifndef DA2_H
@@ -106,7 +107,7 @@ enum {
 typedef enum da2_status {
   DA2_OK = 0,
   DA2_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, budgets out of range */
-  DA2_ERR_UNSUPPORTED = 2,  /* d or bs outside the supported set */
+  DA2_ERR_UNSUPPORTED = 2,  /* d, bs, N or B*H outside the supported set */
   DA2_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
   DA2_ERR_WORKSPACE = 4,    /* ws_bytes smaller than da2_workspace_size */
   DA2_ERR_CUDA = 5,         /* a CUDA call or launch failed */

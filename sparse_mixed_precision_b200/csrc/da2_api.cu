@@ -22,6 +22,9 @@ using namespace da2;
 namespace {
 
 constexpr int kMaxBlocks = 4096;
+constexpr long kMaxHeads = 65535;   // B * H: the stage kernels put the heads on the grid's y axis
+
+bool pct_ok(int p) { return p >= 0 && p <= 100; }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -31,12 +34,15 @@ da2_status check_config(const da2_config* c) {
   if (!c) return DA2_ERR_INVALID_ARG;
   if (c->B <= 0 || c->H <= 0 || c->F <= 0 || c->Hf <= 0 || c->Wf <= 0 || c->ph <= 0 || c->pw <= 0)
     return DA2_ERR_INVALID_ARG;
-  if (c->pct_fp8 < 0 || c->pct_fp4 < 0 || c->pct_mix < 0 || c->pct_fp8 + c->pct_mix + c->pct_fp4 > 100)
+  // each budget on its own first, so that their sums cannot overflow
+  if (!pct_ok(c->pct_fp8) || !pct_ok(c->pct_fp4) || !pct_ok(c->pct_mix) ||
+      c->pct_fp8 + c->pct_mix + c->pct_fp4 > 100)
     return DA2_ERR_INVALID_ARG;
   if (!(c->sm_scale >= 0.0f) || std::isinf(c->sm_scale)) return DA2_ERR_INVALID_ARG;
   if (!(c->adapt_tau >= 0.0f) || std::isinf(c->adapt_tau)) return DA2_ERR_INVALID_ARG;
   if (c->adapt_tau > 0.0f &&
-      (c->pct_fp4_max < c->pct_fp4 || c->pct_fp8 + c->pct_mix + c->pct_fp4_max > 100))
+      (c->pct_fp4_max < c->pct_fp4 || !pct_ok(c->pct_fp4_max) ||
+       c->pct_fp8 + c->pct_mix + c->pct_fp4_max > 100))
     return DA2_ERR_INVALID_ARG;
   if (c->flags & ~(DA2_FLAG_EXPORT_SCORES | DA2_FLAG_NO_MASS_CORRECTION | DA2_FLAG_LAYOUT_BTHD |
                    DA2_FLAG_DEBUG_CANARY | DA2_FLAG_TEST_STALL))
@@ -44,9 +50,12 @@ da2_status check_config(const da2_config* c) {
   if (c->d != 64 && c->d != 128) return DA2_ERR_UNSUPPORTED;
   const long bs = (long)c->ph * c->pw;
   if (bs != 32 && bs != 64 && bs != 128) return DA2_ERR_UNSUPPORTED;
-  const long ny = (c->Hf + c->ph - 1) / c->ph, nx = (c->Wf + c->pw - 1) / c->pw;
+  // in 64-bit steps, each factor bounded before the next product
+  const long ny = ((long)c->Hf + c->ph - 1) / c->ph, nx = ((long)c->Wf + c->pw - 1) / c->pw;
+  if (c->F > kMaxBlocks || ny > kMaxBlocks || nx > kMaxBlocks) return DA2_ERR_UNSUPPORTED;
   const long N = (long)c->F * ny * nx;
   if (N > kMaxBlocks) return DA2_ERR_UNSUPPORTED;
+  if ((long)c->B * c->H > kMaxHeads) return DA2_ERR_UNSUPPORTED;
   if ((long)c->B * c->H * N * N > (1L << 40)) return DA2_ERR_UNSUPPORTED;
   return DA2_OK;
 }

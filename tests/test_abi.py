@@ -214,3 +214,27 @@ def test_binding_refuses_a_bf16_budget():
     with pytest.raises(ValueError, match="bf16"):
         da2.config(scaled(WORKLOADS["tiny"], pct_bf16=5))
     assert da2.config(scaled(WORKLOADS["tiny"], pct_bf16=0)).pct_fp8 == WORKLOADS["tiny"].pct_fp8
+
+
+def test_config_checks_cannot_overflow():
+    # budgets and shapes far outside the supported set are refused before any sum or product
+    # of them can overflow a machine integer
+    L = da2.lib()
+    n = ctypes.c_size_t()
+    w = WORKLOADS["tiny"]
+    big = 2 ** 31 - 1
+
+    def status(**change):
+        cfg = da2.config(scaled(w, **change))
+        return L.da2_workspace_size(ctypes.byref(cfg), ctypes.byref(n))
+    assert status(pct_fp8=big, pct_fp4=1) == 1            # the sum wraps below 100 in 32 bits
+    assert status(pct_fp8=big, pct_fp4=big, pct_mix=2) == 1
+    assert status(pct_fp4=101, pct_fp8=0) == 1
+    assert status(adapt_tau=0.5, pct_fp4_max=big) == 1
+    assert status(Hf=big) == 2                            # Hf + ph - 1 wraps in 32 bits
+    assert status(Wf=big, Hf=1) == 2
+    assert status(F=big, Hf=4, Wf=8) == 2                 # one block per frame, 2^31 - 1 frames
+    assert status(B=2 ** 20, H=2 ** 20) == 2              # B * H * N * N wraps in 64 bits
+    assert status(B=1, H=65535) == 0                      # the largest head count
+    assert status(B=1, H=65536) == 2                      # one more than the grid's y axis
+    assert status(B=3, H=21846) == 2
