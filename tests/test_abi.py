@@ -238,3 +238,41 @@ def test_config_checks_cannot_overflow():
     assert status(B=1, H=65535) == 0                      # the largest head count
     assert status(B=1, H=65536) == 2                      # one more than the grid's y axis
     assert status(B=3, H=21846) == 2
+
+
+def test_plain_c_caller(tmp_path):
+    # the boundary is plain C: a C99 program includes the header, links the library and
+    # sizes a workspace and its views without Python or torch (host-only calls, no GPU)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if gcc is None or not os.path.isdir(cuda_inc):
+        pytest.skip("gcc or the CUDA headers are not installed")
+    src = tmp_path / "caller.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "da2.h"
+int main(void) {
+  da2_config c = {0};
+  c.B = 1; c.H = 2; c.d = 64; c.F = 4; c.Hf = 16; c.Wf = 32; c.ph = 4; c.pw = 8;
+  c.pct_fp8 = 15; c.pct_fp4 = 35;
+  size_t bytes = 0;
+  da2_views v;
+  if (da2_workspace_size(&c, &bytes) != DA2_OK) return 1;
+  if (da2_workspace_views(&c, &v) != DA2_OK) return 2;
+  c.d = 96;
+  if (da2_workspace_size(&c, &bytes) != DA2_ERR_UNSUPPORTED) return 3;
+  printf("%zu %d %d %d %s\n", v.total, v.N, v.n8, v.n4, da2_status_string(DA2_ERR_WORKSPACE));
+  return 0;
+}
+""")
+    libdir = os.path.dirname(da2.LIB_PATH)
+    exe = tmp_path / "caller"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+                    str(src), "-o", str(exe), "-L", libdir, "-l:libda2.so", f"-Wl,-rpath,{libdir}"],
+                   check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    v = da2.workspace_views(da2.config(WORKLOADS["tiny"]))
+    assert [int(x) for x in out[:4]] == [v["total"], v["N"], v["n8"], v["n4"]]
+    assert " ".join(out[4:]) == "workspace too small"
