@@ -1,7 +1,8 @@
 """Python binding of libda2 (the DraftAttention2 hot path on B200, sm_100a).
 
 Argument marshalling only: every step of the path runs in the CUDA library. The names
-follow the C ABI in include/da2.h. Tensors are torch tensors (device memory and streams
+follow the C ABI in include/da2.h. Because that ABI receives bare pointers, the binding
+checks each tensor's dtype, shape, contiguity and device before a call. Tensors are torch tensors (device memory and streams
 come from PyTorch); the library itself allocates no device memory.
 
     cfg = config(workload)                      # da2_config from a synth.Workload
@@ -141,6 +142,51 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def activation_shape(cfg: Config) -> tuple:
+    """Shape of q, k, v and out for a configuration: [B, H, T, d], or [B, T, H, d] with
+    FLAG_LAYOUT_BTHD (T = F * Hf * Wf)."""
+    T = cfg.F * cfg.Hf * cfg.Wf
+    return (cfg.B, T, cfg.H, cfg.d) if cfg.flags & FLAG_LAYOUT_BTHD else (cfg.B, cfg.H, T, cfg.d)
+
+
+def _check_tensors(fn, cfg, acts, bufs=(), host=(), stream=None):
+    """The C ABI takes plain pointers and cannot see a tensor's size, type or placement, so
+    the binding checks them before the call: a wrong tensor raises here instead of sending
+    a kernel out of bounds. acts: (name, tensor) pairs of bf16 activations on the device;
+    host: the same on the host (forward_host); bufs: byte buffers (the workspace) on the
+    device. Every device tensor must sit on the device of the stream the call runs on."""
+    import torch
+    want = activation_shape(cfg)
+    for name, t in list(acts) + list(host):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{fn}: {name} must be a torch.Tensor")
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{fn}: {name} must be bfloat16, not {t.dtype}")
+        if tuple(t.shape) != want:
+            raise ValueError(f"{fn}: {name} has shape {tuple(t.shape)}; the configuration needs {want}")
+    for name, t in list(acts) + list(host) + list(bufs):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{fn}: {name} must be a torch.Tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{fn}: {name} must be contiguous")
+    for name, t in host:
+        if t.device.type != "cpu":
+            raise ValueError(f"{fn}: {name} must be a host tensor, not on {t.device}")
+    dev = list(acts) + list(bufs)
+    for name, t in dev:
+        if t.device.type != "cuda":
+            raise ValueError(f"{fn}: {name} must be a CUDA tensor, not on {t.device}")
+    if dev:
+        sdev = (torch.cuda.current_stream() if stream is None else stream).device
+        for name, t in dev:
+            if t.device != sdev:
+                raise ValueError(f"{fn}: {name} is on {t.device} but the call runs on {sdev}")
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
 def _stream(stream):
     import torch
     s = torch.cuda.current_stream() if stream is None else stream
@@ -160,36 +206,47 @@ def workspace_views(cfg: Config) -> dict:
 
 
 def prepare(cfg, q, k, v, ws, stream=None):
+    _check_tensors("da2_prepare", cfg, (("q", q), ("k", k), ("v", v)), (("ws", ws),), stream=stream)
     _check("da2_prepare", lib().da2_prepare(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
-                                            _ptr(ws), ws.numel(), _stream(stream)))
+                                            _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def draft_select(cfg, ws, stream=None):
-    _check("da2_draft_select", lib().da2_draft_select(ctypes.byref(cfg), _ptr(ws), ws.numel(),
+    _check_tensors("da2_draft_select", cfg, (), (("ws", ws),), stream=stream)
+    _check("da2_draft_select", lib().da2_draft_select(ctypes.byref(cfg), _ptr(ws), _nbytes(ws),
                                                       _stream(stream)))
 
 
 def check_selection(cfg, ws, stream=None):
     """Debug aid: checks the selection's lists and tags in ws (da2_check_selection); a
     violation shows up in get_error."""
-    _check("da2_check_selection", lib().da2_check_selection(ctypes.byref(cfg), _ptr(ws), ws.numel(),
+    _check_tensors("da2_check_selection", cfg, (), (("ws", ws),), stream=stream)
+    _check("da2_check_selection", lib().da2_check_selection(ctypes.byref(cfg), _ptr(ws), _nbytes(ws),
                                                             _stream(stream)))
 
 
 def attention(cfg, ws, out, stream=None):
-    _check("da2_attention", lib().da2_attention(ctypes.byref(cfg), _ptr(ws), ws.numel(),
+    _check_tensors("da2_attention", cfg, (("out", out),), (("ws", ws),), stream=stream)
+    _check("da2_attention", lib().da2_attention(ctypes.byref(cfg), _ptr(ws), _nbytes(ws),
                                                 _ptr(out), _stream(stream)))
 
 
 def forward(cfg, q, k, v, out, ws, stream=None):
+    _check_tensors("da2_forward", cfg, (("q", q), ("k", k), ("v", v), ("out", out)), (("ws", ws),),
+                   stream=stream)
     _check("da2_forward", lib().da2_forward(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
-                                            _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+                                            _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def forward_host(cfg, q_host, k_host, v_host, out_host, dq, dk, dv, dout, ws, stream=None):
+    """q_host, k_host, v_host, out_host: host tensors (pinned for overlapped copies); dq, dk,
+    dv, dout: device staging tensors of the same shape; ws: the device workspace."""
+    _check_tensors("da2_forward_host", cfg, (("dq", dq), ("dk", dk), ("dv", dv), ("dout", dout)),
+                   (("ws", ws),), (("q_host", q_host), ("k_host", k_host), ("v_host", v_host),
+                                   ("out_host", out_host)), stream=stream)
     _check("da2_forward_host", lib().da2_forward_host(
         ctypes.byref(cfg), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(out_host),
-        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dout), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dout), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def forward_noalloc(cfg, q, k, v, out, stream=None):
@@ -197,6 +254,8 @@ def forward_noalloc(cfg, q, k, v, out, stream=None):
     callers that cannot allocate device memory (see da2_forward_noalloc in include/da2.h).
     Calls on one device must not overlap on the GPU: they share that scratch. Its device
     error word is read with get_error(cfg, None)."""
+    _check_tensors("da2_forward_noalloc", cfg, (("q", q), ("k", k), ("v", v), ("out", out)),
+                   stream=stream)
     _check("da2_forward_noalloc", lib().da2_forward_noalloc(
         ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _stream(stream)))
 
@@ -204,8 +263,10 @@ def forward_noalloc(cfg, q, k, v, out, stream=None):
 def get_error(cfg, ws, stream=None) -> int:
     """Reads and clears the workspace's device error word (synchronises the stream).
     ws=None reads the word of forward_noalloc's built-in scratch."""
+    if ws is not None:
+        _check_tensors("da2_get_error", cfg, (), (("ws", ws),), stream=stream)
     word = ctypes.c_uint32()
-    st = lib().da2_get_error(_ptr(ws), 0 if ws is None else ws.numel(), ctypes.byref(cfg),
+    st = lib().da2_get_error(_ptr(ws), 0 if ws is None else _nbytes(ws), ctypes.byref(cfg),
                              _stream(stream), ctypes.byref(word))
     if st not in (0, 6):
         raise DA2Error("da2_get_error", st)

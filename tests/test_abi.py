@@ -276,3 +276,38 @@ int main(void) {
     v = da2.workspace_views(da2.config(WORKLOADS["tiny"]))
     assert [int(x) for x in out[:4]] == [v["total"], v["N"], v["n8"], v["n4"]]
     assert " ".join(out[4:]) == "workspace too small"
+
+
+def test_binding_checks_tensors_before_the_library_sees_them():
+    # the C ABI receives bare pointers, so the binding rejects a tensor of the wrong type,
+    # shape, layout or placement before any call (these raise on a machine without a GPU)
+    import torch
+    w = WORKLOADS["tiny"]
+    cfg = da2.config(w)
+    shape = (w.B, w.H, w.F * w.Hf * w.Wf, w.d)
+    assert da2.activation_shape(cfg) == shape
+    assert da2.activation_shape(da2.config(w, flags=da2.FLAG_LAYOUT_BTHD)) == (shape[0], shape[2], shape[1], shape[3])
+    bf = lambda s=shape: torch.zeros(s, dtype=torch.bfloat16)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="bfloat16"):
+        da2.forward(cfg, bf(), bf(), torch.zeros(shape), bf(), ws)
+    with pytest.raises(ValueError, match="shape"):
+        da2.prepare(cfg, bf(), bf(), bf((w.B, w.H, 100, w.d)), ws)
+    with pytest.raises(ValueError, match="shape"):                 # token-major tensor, head-major config
+        da2.forward(cfg, *(bf((shape[0], shape[2], shape[1], shape[3])) for _ in range(4)), ws)
+    nc = torch.zeros((shape[0], shape[2], shape[1], shape[3]), dtype=torch.bfloat16).transpose(1, 2)
+    with pytest.raises(ValueError, match="contiguous"):
+        da2.forward(cfg, nc, bf(), bf(), bf(), ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):           # host memory handed to a kernel
+        da2.forward(cfg, bf(), bf(), bf(), bf(), ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        da2.draft_select(cfg, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        da2.forward_noalloc(cfg, bf(), bf(), bf(), bf())
+    with pytest.raises(TypeError):
+        da2.attention(cfg, None, bf())
+    # host-buffer call: host tensors on the host, staging buffers and workspace on the device
+    with pytest.raises(ValueError, match="shape"):
+        da2.forward_host(cfg, bf(), bf(), bf(), bf((1, 2, 3, 4)), bf(), bf(), bf(), bf(), ws)
+    with pytest.raises(ValueError, match="dq must be a CUDA tensor"):
+        da2.forward_host(cfg, bf(), bf(), bf(), bf(), bf(), bf(), bf(), bf(), ws)
